@@ -1,0 +1,432 @@
+"""Benchmark of the context-parallel attention hot path on B200.
+
+One step = the whole hot path on the FLUX.1-dev 1024x1024 joint-attention shape
+(B=1, H=24, S=4608, D=128, bf16, QK-normed synthetic inputs):
+  1. Ulysses degree-8 exchange of Q, K and V (sequence-sharded -> head-sharded),
+  2. ring attention over 8 K/V blocks of 576 keys on the head-sharded tensors
+     (blockwise tcgen05 attention writing fp32 partials + LSE, then the LSE merge),
+  3. inverse Ulysses exchange of O.
+Metric: attention TFLOP/s = 4*B*H*S*S*D per step / step time (device time, CUDA
+events, L2 flushed between steps).  Also reported: the dominant kernel's roofline,
+the single-block (ring-1) attention kernel, merge and permute GB/s, the fp64 CPU
+oracle as a baseline, and an end-to-end number through host buffers.
+
+--impl reference times the fp64 CPU oracle (the only reference this project has)
+on a bounded sample of the same workload.  Multi-GPU (torchrun): every rank runs an
+independent replica (the single-GPU path has no data exchange between GPUs).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "flux_1024_ring8_ulysses8"
+METRIC = "attention TFLOP/s (4*B*H*Sq*Skv*D) and % of B200 BF16 peak; merge/permute GB/s"
+UNIT = "TFLOP/s"
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks + throttle reasons sampled every 100 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.samples = []
+        self.proc = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+            return
+        threading.Thread(target=self._read, daemon=True).start()
+        time.sleep(0.8)  # nvidia-smi start-up
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    def stop(self):
+        if self.proc:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = [s for t, s in self.samples if self.t0 and self.t1 and self.t0 - 0.15 <= t <= self.t1 + 0.15]
+        if not rows:
+            rows = [s for _, s in self.samples]
+        mhz, maxmhz, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            parts = [p.strip() for p in r.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                maxmhz = float(parts[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": maxmhz,
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# --------------------------------------------------------------------------- our arm
+
+
+def run_ours(args):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    from context_attention_dit_b200 import binding
+    from context_attention_dit_b200.inputs import WORKLOADS, even_bounds, sha256
+
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    w = WORKLOADS[WORKLOAD]
+    P, B, S, H, D = w.ulysses_degree, w.B, w.S, w.H, w.D
+    n_blocks = len(w.splits[0])
+    q_h, k_h, v_h = w.qkv()
+    sha = {n: sha256(t)[:16] for n, t in zip("qkv", (q_h, k_h, v_h))}
+
+    def seq_shards(x):
+        return x.reshape(B, P, S // P, H, D).permute(1, 0, 2, 3, 4).contiguous()
+
+    xq, xk, xv = (seq_shards(t).to(dev) for t in (q_h, k_h, v_h))  # sequence-sharded inputs
+    Bp, Hp = P * B, H // P
+    bounds = even_bounds(S, n_blocks)
+    parts = torch.empty((n_blocks, Bp, S, Hp, D), dtype=torch.float32, device=dev)
+    lses = torch.empty((n_blocks, Bp, Hp, S), dtype=torch.float32, device=dev)
+    yq, yk, yv = (torch.empty((P, B, S, Hp, D), dtype=torch.bfloat16, device=dev) for _ in range(3))
+    o_h = torch.empty((Bp, S, Hp, D), dtype=torch.bfloat16, device=dev)
+    lse_h = torch.empty((Bp, Hp, S), dtype=torch.float32, device=dev)
+    o_seq = torch.empty((P, B, S // P, H, D), dtype=torch.bfloat16, device=dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+    scale = w.scale
+    flop = w.flop
+    launches_per_step = 3 + 2 + 1
+
+    def step(evs=None):
+        if evs:
+            evs[0].record()
+        binding.ulysses_permute(xq, P, 0, dst=yq)
+        binding.ulysses_permute(xk, P, 0, dst=yk)
+        binding.ulysses_permute(xv, P, 0, dst=yv)
+        if evs:
+            evs[1].record()
+        view = lambda t: t.view(Bp, S, Hp, D)
+        binding.attn_fwd_blocks(view(yq), view(yk), view(yv), bounds, scale=scale, partials=parts, lses=lses)
+        if evs:
+            evs[2].record()
+        binding.attn_merge(parts, lses, out=o_h, out_lse=lse_h)
+        if evs:
+            evs[3].record()
+        binding.ulysses_permute(o_h.view(P, B, S, Hp, D), P, 1, dst=o_seq)
+        if evs:
+            evs[4].record()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert binding.last_device_status() == 0
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.mark_start()
+    for i in range(args.steps):
+        flush.zero_()
+        step(evs[i])
+    torch.cuda.synchronize()
+    clocks.mark_end()
+    if world > 1:
+        dist.barrier()
+    clocks.stop()
+    assert binding.last_device_status() == 0, "device status not OK after timed region"
+
+    step_ms = [e[0].elapsed_time(e[4]) for e in evs]
+    perm_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    attn_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    merge_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    inv_ms = [e[3].elapsed_time(e[4]) for e in evs]
+    total_ms = sum(step_ms)
+    tot = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(tot, op=dist.ReduceOp.MAX)
+    total_ms = float(tot.item())
+
+    # Single-block attention (the FLUX ring-1 case) timed on its own.
+    qd, kd, vd = (t.to(dev) for t in (q_h, k_h, v_h))
+    o1 = torch.empty_like(qd)
+    l1 = torch.empty((B, H, S), dtype=torch.float32, device=dev)
+    r1 = []
+    for i in range(max(args.warmup, 3) + 50):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        binding.attn_fwd(qd, kd, vd, scale=scale, out=o1, lse=l1)
+        b.record()
+        r1.append((a, b))
+    torch.cuda.synchronize()
+    ring1_ms = statistics.mean(a.elapsed_time(b) for a, b in r1[max(args.warmup, 3):])
+
+    # End to end through the public API with host buffers (pinned), per step:
+    # H2D of the sequence-sharded Q/K/V, the hot path, D2H of O.
+    hq, hk, hv = (seq_shards(t).pin_memory() for t in (q_h, k_h, v_h))
+    ho = torch.empty(o_seq.shape, dtype=torch.bfloat16).pin_memory()
+    e2e_steps = max(5, min(50, args.steps // 20))
+    for _ in range(2):
+        xq.copy_(hq, non_blocking=True); xk.copy_(hk, non_blocking=True); xv.copy_(hv, non_blocking=True)
+        step()
+        ho.copy_(o_seq, non_blocking=True)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_steps):
+        xq.copy_(hq, non_blocking=True); xk.copy_(hk, non_blocking=True); xv.copy_(hv, non_blocking=True)
+        step()
+        ho.copy_(o_seq, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    d2h = ho.numel() * ho.element_size()
+
+    if rank == 0:
+        peaks = load_peaks()
+        step_mean = total_ms / args.steps
+        value = world * flop / (total_ms / args.steps * 1e-3) / 1e12
+        attn_mean = statistics.mean(attn_ms)
+        attn_tflops = flop / (attn_mean * 1e-3) / 1e12
+        ring1_tflops = flop / (ring1_ms * 1e-3) / 1e12
+        rows = Bp * Hp * S
+        merge_bytes = n_blocks * rows * (4 * D + 4) + rows * (2 * D + 4)
+        perm_bytes = 3 * 2 * B * S * H * D * 2
+        inv_bytes = 2 * B * S * H * D * 2
+        part_bytes = n_blocks * rows * (4 * D + 4)
+        line = {
+            "metric": METRIC,
+            "value": round(value, 2),
+            "unit": UNIT,
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(step_mean, 4),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) bf16, per-head RMS-normed Q/K; sha256 " + ",".join(
+                f"{k}:{v}" for k, v in sha.items()) + ")",
+            "config": {
+                "workload": ("FLUX.1-dev 1024x1024 joint attention B1 H24 S4608 D128: Ulysses-8 exchange of Q/K/V, "
+                             "ring-8 blockwise attention (8 x 576 keys) + LSE merge, inverse exchange of O"),
+                "global_batch": world * B, "seq_len": S, "heads": H, "head_dim": D,
+                "ulysses_degree": P, "ring_degree": n_blocks,
+                "parallelism": f"replicas x{world} (single-GPU simulated degrees)",
+                "l2": "flushed between timed steps (write of %d MiB > L2)" % (flush.numel() >> 20),
+            },
+            "roofline": {
+                "kernel": "attn_fwd_sm100 (8 ring blocks in one launch)",
+                "bound": "tensor",
+                "achieved": round(attn_tflops, 2),
+                "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s",
+                "frac": round(attn_tflops / peaks["bf16_tflops"], 4),
+                "frac_of_sustained": round(attn_tflops / peaks["bf16_tflops_sustained"], 4)
+                if peaks["bf16_tflops_sustained"] else None,
+                "frac_of_spec_2250": round(attn_tflops / 2250.0, 4),
+                "peak_source": peaks["source"] + " (burst bf16 GEMM)",
+                "flop_per_launch": flop,
+                "traffic": None,
+            },
+            "kernels": {
+                "attn_ring1_tflops": round(ring1_tflops, 2),
+                "attn_ring1_ms": round(ring1_ms, 4),
+                "attn_ring8_ms": round(attn_mean, 4),
+                "attn_ring8_partial_bytes": part_bytes,
+                "merge_ms": round(statistics.mean(merge_ms), 4),
+                "merge_gbs": round(merge_bytes / (statistics.mean(merge_ms) * 1e-3) / 1e9, 1),
+                "permute_qkv_ms": round(statistics.mean(perm_ms), 4),
+                "permute_qkv_gbs": round(perm_bytes / (statistics.mean(perm_ms) * 1e-3) / 1e9, 1),
+                "permute_inv_ms": round(statistics.mean(inv_ms), 4),
+                "permute_inv_gbs": round(inv_bytes / (statistics.mean(inv_ms) * 1e-3) / 1e9, 1),
+                "hbm_peak_gbs": peaks["hbm_gbs"],
+            },
+            "e2e": {"value": round(world * flop / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks.summary(),
+        }
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_budget)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# --------------------------------------------------------------------------- the oracle
+
+
+def _oracle_step(q, k, v, scale, bounds, rows):
+    """One oracle pass: ring attention (per block + LSE merge) for the sampled query rows."""
+    import oracle
+
+    return oracle.ring(q[:, rows], k, v, scale, bounds)
+
+
+def _threads_used():
+    try:
+        from threadpoolctl import threadpool_info
+
+        info = threadpool_info()
+        return max((i.get("num_threads", 1) for i in info), default=1)
+    except Exception:
+        return 1
+
+
+def _sample_rows(S, n):
+    import numpy as np
+
+    return sorted(np.random.default_rng(0).choice(S, size=n, replace=False).tolist())
+
+
+def cpu_baseline(budget_s: float = 15.0):
+    """Time the fp64 oracle as it stands on a bounded sample of the workload (rank 0 only)."""
+    from context_attention_dit_b200.inputs import WORKLOADS, even_bounds
+
+    w = WORKLOADS[WORKLOAD]
+    q, k, v = w.qkv()
+    bounds = even_bounds(w.S, len(w.splits[0]))
+    # calibrate the sample size on 64 rows, then size it to the budget
+    t0 = time.time()
+    _oracle_step(q, k, v, w.scale, bounds, _sample_rows(w.S, 64))
+    per_row = (time.time() - t0) / 64
+    n_rows = int(max(64, min(w.S, budget_s / max(per_row, 1e-6))))
+    rows = _sample_rows(w.S, n_rows)
+    t0 = time.time()
+    _oracle_step(q, k, v, w.scale, bounds, rows)
+    dt = time.time() - t0
+    flop = 4 * w.B * w.H * n_rows * w.S * w.D
+    return {"value": round(flop / dt / 1e12, 6), "unit": UNIT, "cores": _threads_used(), "kind": "oracle",
+            "sample": f"ring-8 attention + LSE merge (fp64 numpy) for {n_rows} of {w.S} query rows, all 24 heads, "
+                      f"{dt:.1f} s", "seconds": round(dt, 2)}
+
+
+def run_reference(args):
+    world, rank, _ = dist_setup()
+    if rank != 0:
+        return
+    from context_attention_dit_b200.inputs import WORKLOADS, even_bounds
+
+    w = WORKLOADS[WORKLOAD]
+    q, k, v = w.qkv()
+    bounds = even_bounds(w.S, len(w.splits[0]))
+    budget_per_step = max(0.05, args.ref_budget / max(1, args.steps + args.warmup))
+    t0 = time.time()
+    _oracle_step(q, k, v, w.scale, bounds, _sample_rows(w.S, 16))
+    per_row = (time.time() - t0) / 16
+    n_rows = int(max(1, min(w.S, budget_per_step / max(per_row, 1e-6))))
+    rows = _sample_rows(w.S, n_rows)
+    for _ in range(args.warmup):
+        _oracle_step(q, k, v, w.scale, bounds, rows)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.time()
+        _oracle_step(q, k, v, w.scale, bounds, rows)
+        times.append(time.time() - t0)
+    total = sum(times)
+    flop = 4 * w.B * w.H * n_rows * w.S * w.D
+    value = flop * args.steps / total / 1e12
+    line = {
+        "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": "FLUX.1-dev 1024x1024 joint attention B1 H24 S4608 D128, ring-8 + LSE merge "
+                               f"(fp64 CPU oracle, {n_rows} sampled query rows per step)"},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": _threads_used(), "kind": "oracle",
+                         "sample": f"{n_rows} of {w.S} query rows per step, all heads, 8 K/V blocks + merge"},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--ref-budget", type=float, default=90.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,257 @@
+"""Thin ctypes binding of libcpattn.so (argument marshalling only).
+
+Torch tensors supply device memory and the current stream; every step of the
+computation runs in the library's CUDA kernels.  The binding checks what the
+C ABI cannot see, mirroring the attention dispatcher's checks ("Attention
+backends", section "Checks": query/key/value on one device, matching dtypes,
+usually bfloat16, and valid shapes) and raises ``ValueError``.  A non-OK status
+from the library raises ``RuntimeError`` with the status name.  There is no
+fallback: if the library is missing or fails to load, every call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libcpattn.so")
+
+CP_OK = 0
+CP_ERR_INVALID_ARG = -1
+CP_ERR_UNSUPPORTED = -2
+CP_ERR_NOT_DIVISIBLE = -3
+CP_ERR_MISALIGNED = -4
+CP_ERR_CUDA = -5
+CP_ERR_TIMEOUT = -6
+CP_BF16 = 0
+CP_F32 = 1
+CP_MAX_CHUNKS = 64
+
+EXPORTS = (
+    "cp_attn_fwd", "cp_attn_fwd_blocks", "cp_attn_merge", "cp_ring_sim_workspace_size", "cp_ring_sim", "cp_ulysses_permute",
+    "cp_ring_bounds", "cp_last_device_status", "cp_status_string", "cp_version",
+)
+
+_lib = None
+
+
+class CpError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+def load() -> ctypes.CDLL:
+    """Load libcpattn.so (built in-tree); raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"libcpattn.so not built at {LIB_PATH}; run python -m context_attention_dit_b200.build")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    ip = ctypes.POINTER(ctypes.c_int)
+    lib.cp_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
+    lib.cp_attn_fwd_blocks.argtypes = [vp, vp, vp, ip, i, vp, vp, i, i, i, i, i, f, vp]
+    lib.cp_attn_merge.argtypes = [vp, vp, i, vp, vp, i, i, i, i, i, vp]
+    lib.cp_ring_sim_workspace_size.argtypes = [i, i, i, i, i]
+    lib.cp_ring_sim_workspace_size.restype = sz
+    lib.cp_ring_sim.argtypes = [vp, vp, vp, ip, i, vp, vp, i, i, i, i, i, f, i, vp, sz, vp]
+    lib.cp_ulysses_permute.argtypes = [vp, vp, i, i, i, i, i, i, i, vp]
+    lib.cp_ring_bounds.argtypes = [i, i, i, ip]
+    lib.cp_last_device_status.argtypes = [vp]
+    lib.cp_status_string.argtypes = [i]
+    lib.cp_status_string.restype = ctypes.c_char_p
+    lib.cp_version.argtypes = []
+    for name in ("cp_attn_fwd", "cp_attn_fwd_blocks", "cp_attn_merge", "cp_ring_sim", "cp_ulysses_permute", "cp_ring_bounds",
+                 "cp_last_device_status"):
+        getattr(lib, name).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load().cp_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != CP_OK:
+        raise CpError(status, where)
+
+
+def _stream(t: torch.Tensor) -> int:
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _out_code(dtype) -> int:
+    if dtype == torch.bfloat16:
+        return CP_BF16
+    if dtype == torch.float32:
+        return CP_F32
+    raise ValueError(f"output dtype must be bfloat16 or float32, got {dtype}")
+
+
+def _check_qkv(q, k, v):
+    for name, t in (("query", q), ("key", k), ("value", v)):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if t.dtype != torch.bfloat16:
+            raise ValueError(f"{name} must be bfloat16, got {t.dtype}")
+        if t.dim() != 4:
+            raise ValueError(f"{name} must be 4-D (batch, seq, heads, head_dim), got {tuple(t.shape)}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous (BSHD)")
+    if not (q.device == k.device == v.device):
+        raise ValueError("query, key and value must be on the same device")
+    B, Sq, H, D = q.shape
+    if k.shape != v.shape or k.shape[0] != B or k.shape[2] != H or k.shape[3] != D:
+        raise ValueError(f"incompatible shapes q{tuple(q.shape)} k{tuple(k.shape)} v{tuple(v.shape)}")
+    return B, Sq, k.shape[1], H, D
+
+
+def attn_fwd(q, k, v, scale: Optional[float] = None, out_dtype=torch.bfloat16, out=None, lse=None,
+             want_lse: bool = True):
+    """Attention of q over one K/V block; returns ``(out [B,Sq,H,D], lse [B,H,Sq] fp32)``."""
+    B, Sq, Skv, H, D = _check_qkv(q, k, v)
+    code = _out_code(out_dtype)
+    scale = float(D ** -0.5 if scale is None else scale)
+    if out is None:
+        out = torch.empty((B, Sq, H, D), dtype=out_dtype, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
+    st = load().cp_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Sq, Skv, D, scale, code,
+                            ctypes.c_void_p(_stream(q)))
+    _check(st, "cp_attn_fwd")
+    return out, lse
+
+
+def attn_fwd_blocks(q, k, v, chunk_bounds: Sequence[int], scale: Optional[float] = None, partials=None,
+                    lses=None):
+    """Attention of q over each K/V block ``[c_r, c_{r+1})`` in one launch (no merge).
+
+    Returns fp32 ``(partials [n,B,Sq,H,D], lses [n,B,H,Sq])``, the inputs of :func:`attn_merge`.
+    """
+    B, Sq, Skv, H, D = _check_qkv(q, k, v)
+    scale = float(D ** -0.5 if scale is None else scale)
+    n = len(chunk_bounds) - 1
+    if n < 1:
+        raise ValueError("chunk_bounds needs at least two entries")
+    bounds = (ctypes.c_int * (n + 1))(*[int(c) for c in chunk_bounds])
+    if partials is None:
+        partials = torch.empty((n, B, Sq, H, D), dtype=torch.float32, device=q.device)
+    if lses is None:
+        lses = torch.empty((n, B, H, Sq), dtype=torch.float32, device=q.device)
+    st = load().cp_attn_fwd_blocks(_ptr(q), _ptr(k), _ptr(v), bounds, n, _ptr(partials), _ptr(lses), B, H, Sq, Skv,
+                                   D, scale, ctypes.c_void_p(_stream(q)))
+    _check(st, "cp_attn_fwd_blocks")
+    return partials, lses
+
+
+def attn_merge(partials, lses, out_dtype=torch.bfloat16, out=None, out_lse=None):
+    """Merge fp32 partials ``[n,B,Sq,H,D]`` with LSEs ``[n,B,H,Sq]``; returns ``(out, lse)``."""
+    if partials.dtype != torch.float32 or lses.dtype != torch.float32:
+        raise ValueError("partials and lses must be float32")
+    if not (partials.is_cuda and lses.is_cuda) or partials.device != lses.device:
+        raise ValueError("partials and lses must be CUDA tensors on one device")
+    if not (partials.is_contiguous() and lses.is_contiguous()):
+        raise ValueError("partials and lses must be contiguous")
+    n, B, Sq, H, D = partials.shape
+    if tuple(lses.shape) != (n, B, H, Sq):
+        raise ValueError(f"lses shape {tuple(lses.shape)} != {(n, B, H, Sq)}")
+    code = _out_code(out_dtype)
+    if out is None:
+        out = torch.empty((B, Sq, H, D), dtype=out_dtype, device=partials.device)
+    if out_lse is None:
+        out_lse = torch.empty((B, H, Sq), dtype=torch.float32, device=partials.device)
+    st = load().cp_attn_merge(_ptr(partials), _ptr(lses), n, _ptr(out), _ptr(out_lse), B, H, Sq, D, code,
+                              ctypes.c_void_p(_stream(partials)))
+    _check(st, "cp_attn_merge")
+    return out, out_lse
+
+
+def ring_workspace_size(n_chunks: int, B: int, H: int, Sq: int, D: int) -> int:
+    return int(load().cp_ring_sim_workspace_size(n_chunks, B, H, Sq, D))
+
+
+def ring_sim(q, k, v, chunk_bounds: Sequence[int], scale: Optional[float] = None, out_dtype=torch.bfloat16,
+             workspace=None, out=None, out_lse=None):
+    """Ring / ring-anything attention over K/V blocks ``[c_r, c_{r+1})``; returns ``(out, lse, workspace)``."""
+    B, Sq, Skv, H, D = _check_qkv(q, k, v)
+    code = _out_code(out_dtype)
+    scale = float(D ** -0.5 if scale is None else scale)
+    n = len(chunk_bounds) - 1
+    if n < 1:
+        raise ValueError("chunk_bounds needs at least two entries")
+    bounds = (ctypes.c_int * (n + 1))(*[int(c) for c in chunk_bounds])
+    need = ring_workspace_size(n, B, H, Sq, D)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if out is None:
+        out = torch.empty((B, Sq, H, D), dtype=out_dtype, device=q.device)
+    if out_lse is None:
+        out_lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
+    st = load().cp_ring_sim(_ptr(q), _ptr(k), _ptr(v), bounds, n, _ptr(out), _ptr(out_lse), B, H, Sq, Skv, D, scale,
+                            code, _ptr(workspace), ws_bytes, ctypes.c_void_p(_stream(q)))
+    _check(st, "cp_ring_sim")
+    return out, out_lse, workspace
+
+
+def ring_workspace_views(workspace, n: int, B: int, H: int, Sq: int, D: int):
+    """Views of the per-block fp32 partials ``[n,B,Sq,H,D]`` and LSEs ``[n,B,H,Sq]`` in a ring workspace."""
+    rows = B * H * Sq
+    pbytes = (n * rows * D * 4 + 255) // 256 * 256
+    parts = workspace[: n * rows * D * 4].view(torch.float32).view(n, B, Sq, H, D)
+    lses = workspace[pbytes: pbytes + n * rows * 4].view(torch.float32).view(n, B, H, Sq)
+    return parts, lses
+
+
+def ulysses_permute(src, degree: int, direction: int, dst=None):
+    """Ulysses exchange.  direction 0: ``[P,B,S/P,H,D] -> [P,B,S,H/P,D]``; direction 1: the inverse."""
+    if not src.is_cuda or not src.is_contiguous():
+        raise ValueError("src must be a contiguous CUDA tensor")
+    if src.element_size() not in (2, 4):
+        raise ValueError("src elements must be 2 or 4 bytes")
+    P = int(degree)
+    if src.dim() != 5 or src.shape[0] != P:
+        raise ValueError(f"src must be 5-D with leading dim {P}, got {tuple(src.shape)}")
+    if direction == 0:
+        _, B, Sp, H, D = src.shape
+        S = Sp * P
+        if H % P:
+            raise ValueError(f"heads {H} not divisible by degree {P}")
+        shape = (P, B, S, H // P, D)
+    elif direction == 1:
+        _, B, S, Hp, D = src.shape
+        H = Hp * P
+        if S % P:
+            raise ValueError(f"sequence {S} not divisible by degree {P}")
+        shape = (P, B, S // P, H, D)
+    else:
+        raise ValueError("direction must be 0 or 1")
+    if dst is None:
+        dst = torch.empty(shape, dtype=src.dtype, device=src.device)
+    st = load().cp_ulysses_permute(_ptr(src), _ptr(dst), P, B, S, H, D, direction, src.element_size(),
+                                   ctypes.c_void_p(_stream(src)))
+    _check(st, "cp_ulysses_permute")
+    return dst
+
+
+def ring_bounds(S: int, n: int, anything: bool = False):
+    """Block bounds of a ring of ``n`` over ``S`` rows (host only)."""
+    out = (ctypes.c_int * (n + 1))()
+    _check(load().cp_ring_bounds(int(S), int(n), 1 if anything else 0, out), "cp_ring_bounds")
+    return list(out)
+
+
+def last_device_status(stream=None) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return int(load().cp_last_device_status(ctypes.c_void_p(s.cuda_stream)))

@@ -1,0 +1,341 @@
+// cpattn.cu - the C ABI of libcpattn.so (declared in include/cpattn.h).
+//
+// Host side only: argument checks (all before any CUDA call, so a bad argument never
+// launches anything), TMA descriptor encoding, and kernel launches on the caller's
+// stream.  Every step of the computation runs in the kernels included below.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/cpattn.h"
+#include "attn_fwd_sm100.cuh"
+#include "lse_merge.cuh"
+#include "ulysses_permute.cuh"
+
+using namespace cpattn;
+
+static_assert(kMaxChunks == CP_MAX_CHUNKS, "chunk limit mismatch");
+
+// Device status word: kernels record CP_ERR_TIMEOUT here when a bounded wait runs out.
+__device__ int g_cp_status = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool init = false;
+  int num_sms = 0;
+  int* status = nullptr;  // device address of g_cp_status
+  bool attn_attr_set[2] = {false, false};
+};
+
+std::mutex g_mutex;
+DeviceInfo g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+cp_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CP_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.init) {
+    if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return CP_ERR_CUDA;
+    void* sym = nullptr;
+    if (cudaGetSymbolAddress(&sym, g_cp_status) != cudaSuccess) return CP_ERR_CUDA;
+    d.status = static_cast<int*>(sym);
+    if (!g_encode) {
+      cudaDriverEntryPointQueryResult q;
+      void* fn = nullptr;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || !fn)
+        return CP_ERR_CUDA;
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    d.init = true;
+  }
+  *out = &d;
+  return CP_OK;
+}
+
+// 4-D map over a BSHD bf16 tensor: dims (D, H, S, B), box (64, 1, 128, 1), 128B swizzle.
+// Rows past S read as zeros.
+cp_status make_bshd_map(CUtensorMap* m, const void* base, int B, int S, int H, int D) {
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(S),
+                        static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2,
+                           static_cast<cuuint64_t>(S) * H * D * 2};
+  cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(kBM), 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? CP_OK : CP_ERR_CUDA;
+}
+
+cp_status check_attn_args(const void* q, const void* k, const void* v, const void* out, const float* lse, int B,
+                          int H, int Sq, int Skv, int D, float scale, cp_dtype out_dtype) {
+  if (B < 0 || H < 0 || Sq < 0 || Skv < 0) return CP_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return CP_ERR_UNSUPPORTED;
+  if (out_dtype != CP_BF16 && out_dtype != CP_F32) return CP_ERR_INVALID_ARG;
+  if (!(std::isfinite(scale) && scale > 0.f)) return CP_ERR_INVALID_ARG;
+  if (B == 0 || H == 0 || Sq == 0) return CP_OK;
+  if (!q || !out) return CP_ERR_INVALID_ARG;
+  if (Skv > 0 && (!k || !v)) return CP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(out) || (Skv > 0 && (!aligned16(k) || !aligned16(v))) ||
+      (lse && !aligned16(lse)))
+    return CP_ERR_MISALIGNED;
+  // 32-bit limits: TMA coordinates, item counts.
+  const long long n_qt = (Sq + kBM - 1) / kBM;
+  if (static_cast<long long>(B) * H * n_qt * kMaxChunks >= (1LL << 31)) return CP_ERR_UNSUPPORTED;
+  return CP_OK;
+}
+
+// Launch the attention kernel over n_chunks K/V blocks given by `bounds` (host array).
+cp_status launch_attn(const void* q, const void* k, const void* v, const int* bounds, int n_chunks, void* out,
+                      int out_f32, long long out_chunk_stride, float* lse, long long lse_chunk_stride, int B, int H,
+                      int Sq, int Skv, int D, float scale, cudaStream_t stream) {
+  DeviceInfo* dev = nullptr;
+  cp_status st = device_info(&dev);
+  if (st != CP_OK) return st;
+  AttnParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.B = B;
+  p.H = H;
+  p.Sq = Sq;
+  p.n_chunks = n_chunks;
+  p.n_qt = (Sq + kBM - 1) / kBM;
+  p.total_items = B * H * n_chunks * p.n_qt;
+  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.out = out;
+  p.out_f32 = out_f32;
+  p.out_chunk_stride = out_chunk_stride;
+  p.lse = lse;
+  p.lse_chunk_stride = lse_chunk_stride;
+  p.status = dev->status;
+  for (int i = 0; i <= n_chunks; ++i) p.bounds[i] = bounds[i];
+
+  CUtensorMap tq, tk, tv;
+  // A map needs at least one row; with Skv == 0 every block is empty and K/V are never read.
+  const int kv_rows = Skv > 0 ? Skv : 1;
+  const void* kp = Skv > 0 ? k : q;
+  const void* vp = Skv > 0 ? v : q;
+  if (make_bshd_map(&tq, q, B, Sq, H, D) != CP_OK || make_bshd_map(&tk, kp, B, Skv > 0 ? kv_rows : Sq, H, D) != CP_OK ||
+      make_bshd_map(&tv, vp, B, Skv > 0 ? kv_rows : Sq, H, D) != CP_OK)
+    return CP_ERR_CUDA;
+
+  const int grid = p.total_items < dev->num_sms ? p.total_items : dev->num_sms;
+  if (D == 128) {
+    using L = AttnSmem<128>;
+    if (!dev->attn_attr_set[1]) {
+      if (cudaFuncSetAttribute(attn_fwd_sm100_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               L::kRequest) != cudaSuccess)
+        return CP_ERR_CUDA;
+      dev->attn_attr_set[1] = true;
+    }
+    attn_fwd_sm100_kernel<128><<<grid, kAttnThreads, L::kRequest, stream>>>(tq, tk, tv, p);
+  } else {
+    using L = AttnSmem<64>;
+    if (!dev->attn_attr_set[0]) {
+      if (cudaFuncSetAttribute(attn_fwd_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               L::kRequest) != cudaSuccess)
+        return CP_ERR_CUDA;
+      dev->attn_attr_set[0] = true;
+    }
+    attn_fwd_sm100_kernel<64><<<grid, kAttnThreads, L::kRequest, stream>>>(tq, tk, tv, p);
+  }
+  return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+}
+
+cp_status launch_merge(const float* partials, const float* lses, int n, void* out, float* out_lse, int B, int H,
+                       int Sq, int D, cp_dtype out_dtype, cudaStream_t stream) {
+  const long long rows = static_cast<long long>(B) * H * Sq;
+  const long long part_stride = rows * D;
+  const long long lse_stride = rows;
+  const long long blocks = (rows + kMergeThreads / 32 - 1) / (kMergeThreads / 32);
+  if (blocks >= (1LL << 31)) return CP_ERR_UNSUPPORTED;
+  const dim3 grid(static_cast<unsigned>(blocks));
+  if (D == 128) {
+    if (out_dtype == CP_BF16)
+      lse_merge_kernel<128, true><<<grid, kMergeThreads, 0, stream>>>(partials, lses, n, out, out_lse, H, Sq, rows,
+                                                                      part_stride, lse_stride);
+    else
+      lse_merge_kernel<128, false><<<grid, kMergeThreads, 0, stream>>>(partials, lses, n, out, out_lse, H, Sq, rows,
+                                                                       part_stride, lse_stride);
+  } else {
+    if (out_dtype == CP_BF16)
+      lse_merge_kernel<64, true><<<grid, kMergeThreads, 0, stream>>>(partials, lses, n, out, out_lse, H, Sq, rows,
+                                                                     part_stride, lse_stride);
+    else
+      lse_merge_kernel<64, false><<<grid, kMergeThreads, 0, stream>>>(partials, lses, n, out, out_lse, H, Sq, rows,
+                                                                      part_stride, lse_stride);
+  }
+  return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+}
+
+cp_status check_bounds(const int* chunk_bounds, int n_chunks, int Skv) {
+  if (n_chunks < 1 || !chunk_bounds) return CP_ERR_INVALID_ARG;
+  if (n_chunks > CP_MAX_CHUNKS) return CP_ERR_UNSUPPORTED;
+  if (Skv < 0) return CP_ERR_INVALID_ARG;
+  if (chunk_bounds[0] != 0 || chunk_bounds[n_chunks] != Skv) return CP_ERR_INVALID_ARG;
+  for (int i = 0; i < n_chunks; ++i)
+    if (chunk_bounds[i] > chunk_bounds[i + 1]) return CP_ERR_INVALID_ARG;
+  return CP_OK;
+}
+
+inline size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+}  // namespace
+
+extern "C" {
+
+int cp_version(void) { return 100; }
+
+const char* cp_status_string(cp_status s) {
+  switch (s) {
+    case CP_OK: return "CP_OK";
+    case CP_ERR_INVALID_ARG: return "CP_ERR_INVALID_ARG: invalid argument";
+    case CP_ERR_UNSUPPORTED: return "CP_ERR_UNSUPPORTED: unsupported size or head_dim";
+    case CP_ERR_NOT_DIVISIBLE: return "CP_ERR_NOT_DIVISIBLE: sequence or heads not divisible by the degree";
+    case CP_ERR_MISALIGNED: return "CP_ERR_MISALIGNED: device pointer not 16-byte aligned";
+    case CP_ERR_CUDA: return "CP_ERR_CUDA: CUDA runtime or driver error";
+    case CP_ERR_TIMEOUT: return "CP_ERR_TIMEOUT: a device-side wait ran out";
+  }
+  return "unknown cp_status";
+}
+
+cp_status cp_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H, int Sq,
+                      int Skv, int D, float scale, cp_dtype out_dtype, void* stream) {
+  cp_status st = check_attn_args(q, k, v, out, lse, B, H, Sq, Skv, D, scale, out_dtype);
+  if (st != CP_OK || B == 0 || H == 0 || Sq == 0) return st;
+  const int bounds[2] = {0, Skv};
+  return launch_attn(q, k, v, bounds, 1, out, out_dtype == CP_F32 ? 1 : 0, 0, lse, 0, B, H, Sq, Skv, D, scale,
+                     static_cast<cudaStream_t>(stream));
+}
+
+cp_status cp_attn_merge(const float* partials, const float* lses, int n_chunks, void* out, float* out_lse, int B,
+                        int H, int Sq, int D, cp_dtype out_dtype, void* stream) {
+  if (B < 0 || H < 0 || Sq < 0) return CP_ERR_INVALID_ARG;
+  if (n_chunks < 1 || n_chunks > CP_MAX_CHUNKS) return n_chunks < 1 ? CP_ERR_INVALID_ARG : CP_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128) return CP_ERR_UNSUPPORTED;
+  if (out_dtype != CP_BF16 && out_dtype != CP_F32) return CP_ERR_INVALID_ARG;
+  if (B == 0 || H == 0 || Sq == 0) return CP_OK;
+  if (!partials || !lses || !out) return CP_ERR_INVALID_ARG;
+  if (!aligned16(partials) || !aligned16(lses) || !aligned16(out) || (out_lse && !aligned16(out_lse)))
+    return CP_ERR_MISALIGNED;
+  return launch_merge(partials, lses, n_chunks, out, out_lse, B, H, Sq, D, out_dtype,
+                      static_cast<cudaStream_t>(stream));
+}
+
+size_t cp_ring_sim_workspace_size(int n_chunks, int B, int H, int Sq, int D) {
+  if (n_chunks <= 1 || B <= 0 || H <= 0 || Sq <= 0 || D <= 0) return 0;
+  const size_t rows = static_cast<size_t>(B) * H * Sq;
+  return round256(static_cast<size_t>(n_chunks) * rows * D * sizeof(float)) +
+         round256(static_cast<size_t>(n_chunks) * rows * sizeof(float));
+}
+
+cp_status cp_attn_fwd_blocks(const void* q, const void* k, const void* v, const int* chunk_bounds, int n_chunks,
+                             float* partials, float* lses, int B, int H, int Sq, int Skv, int D, float scale,
+                             void* stream) {
+  cp_status st = check_bounds(chunk_bounds, n_chunks, Skv);
+  if (st != CP_OK) return st;
+  st = check_attn_args(q, k, v, partials, lses, B, H, Sq, Skv, D, scale, CP_F32);
+  if (st != CP_OK || B == 0 || H == 0 || Sq == 0) return st;
+  if (!lses) return CP_ERR_INVALID_ARG;
+  const long long rows = static_cast<long long>(B) * H * Sq;
+  return launch_attn(q, k, v, chunk_bounds, n_chunks, partials, 1, rows * D, lses, rows, B, H, Sq, Skv, D, scale,
+                     static_cast<cudaStream_t>(stream));
+}
+
+cp_status cp_ring_sim(const void* q, const void* k, const void* v, const int* chunk_bounds, int n_chunks, void* out,
+                      float* out_lse, int B, int H, int Sq, int Skv, int D, float scale, cp_dtype out_dtype,
+                      void* workspace, size_t ws_bytes, void* stream) {
+  cp_status st = check_bounds(chunk_bounds, n_chunks, Skv);
+  if (st != CP_OK) return st;
+  st = check_attn_args(q, k, v, out, out_lse, B, H, Sq, Skv, D, scale, out_dtype);
+  if (st != CP_OK || B == 0 || H == 0 || Sq == 0) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (n_chunks == 1)
+    return launch_attn(q, k, v, chunk_bounds, 1, out, out_dtype == CP_F32 ? 1 : 0, 0, out_lse, 0, B, H, Sq, Skv, D,
+                       scale, s);
+  const size_t need = cp_ring_sim_workspace_size(n_chunks, B, H, Sq, D);
+  if (!workspace || ws_bytes < need) return CP_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return CP_ERR_MISALIGNED;
+  const long long rows = static_cast<long long>(B) * H * Sq;
+  float* partials = static_cast<float*>(workspace);
+  float* lses = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                         round256(static_cast<size_t>(n_chunks) * rows * D * sizeof(float)));
+  st = launch_attn(q, k, v, chunk_bounds, n_chunks, partials, 1, rows * D, lses, rows, B, H, Sq, Skv, D, scale, s);
+  if (st != CP_OK) return st;
+  return launch_merge(partials, lses, n_chunks, out, out_lse, B, H, Sq, D, out_dtype, s);
+}
+
+cp_status cp_ulysses_permute(const void* src, void* dst, int degree, int B, int S, int H, int D, int direction,
+                             int elem_bytes, void* stream) {
+  if (degree < 1 || B < 0 || S < 0 || H < 0 || D < 0) return CP_ERR_INVALID_ARG;
+  if (direction != 0 && direction != 1) return CP_ERR_INVALID_ARG;
+  if (elem_bytes != 2 && elem_bytes != 4) return CP_ERR_UNSUPPORTED;
+  if (S % degree != 0 || H % degree != 0) return CP_ERR_NOT_DIVISIBLE;
+  if (B == 0 || S == 0 || H == 0 || D == 0) return CP_OK;
+  if (!src || !dst) return CP_ERR_INVALID_ARG;
+  if (!aligned16(src) || !aligned16(dst)) return CP_ERR_MISALIGNED;
+  const long long row_bytes = static_cast<long long>(H) * D * elem_bytes;
+  const long long piece_bytes = row_bytes / degree;
+  const long long total = static_cast<long long>(B) * S * row_bytes;
+  const char* s0 = static_cast<const char*>(src);
+  const char* d0 = static_cast<const char*>(dst);
+  if (s0 < d0 + total && d0 < s0 + total) return CP_ERR_INVALID_ARG;  // overlap
+  if (static_cast<long long>(degree) * B > 65535 || row_bytes / 2 >= (1LL << 31)) return CP_ERR_UNSUPPORTED;
+  DeviceInfo* dev = nullptr;
+  cp_status st = device_info(&dev);
+  if (st != CP_OK) return st;
+  const int Sp = S / degree;
+  const unsigned gy = static_cast<unsigned>(Sp < 65535 ? Sp : 65535);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  auto launch = [&](auto tag) {
+    using V = decltype(tag);
+    const int row_vecs = static_cast<int>(row_bytes / sizeof(V));
+    const int piece_vecs = static_cast<int>(piece_bytes / sizeof(V));
+    const dim3 grid((row_vecs + kPermuteThreads - 1) / kPermuteThreads, gy, degree * B);
+    ulysses_permute_kernel<V><<<grid, kPermuteThreads, 0, cs>>>(static_cast<const V*>(src), static_cast<V*>(dst),
+                                                                degree, B, Sp, row_vecs, piece_vecs, direction);
+  };
+  if (piece_bytes % 16 == 0)
+    launch(uint4{});
+  else if (piece_bytes % 8 == 0)
+    launch(uint2{});
+  else if (piece_bytes % 4 == 0)
+    launch(uint32_t{});
+  else
+    launch(uint16_t{});
+  return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+}
+
+cp_status cp_ring_bounds(int S, int n, int anything, int* bounds_out) {
+  if (S < 0 || n < 1 || !bounds_out) return CP_ERR_INVALID_ARG;
+  if (!anything && S % n != 0) return CP_ERR_NOT_DIVISIBLE;
+  const int base = S / n, extra = S % n;
+  bounds_out[0] = 0;
+  for (int i = 0; i < n; ++i) bounds_out[i + 1] = bounds_out[i] + base + (i < extra ? 1 : 0);
+  return CP_OK;
+}
+
+cp_status cp_last_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return CP_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_cp_status, sizeof(int)) != cudaSuccess) return CP_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_cp_status, &zero, sizeof(int)) != cudaSuccess) return CP_ERR_CUDA;
+  }
+  return static_cast<cp_status>(v);
+}
+
+}  // extern "C"

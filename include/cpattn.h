@@ -1,0 +1,183 @@
+/*
+ * cpattn.h - C ABI of libcpattn.so: the single-GPU hot path of context-parallel
+ * attention for diffusion transformers, hand-written for B200 (sm_100a).
+ *
+ * What is computed (sources are web pages on diffusers' context parallelism):
+ *   - "Attention backends", section "Available backends": the default backend is
+ *     scaled_dot_product_attention, i.e. non-causal softmax(Q K^T * scale) V over
+ *     (batch, seq, heads, head_dim) tensors (section "Checks" uses (1, 10, 8, 64)).
+ *   - "Context parallelism", section "Ring Attention": K/V blocks are attended one
+ *     after another; section "Ring Anything Attention": blocks of unequal length.
+ *   - "Parallelism" (API page), ContextParallelConfig.convert_to_fp32: each block's
+ *     output and LSE are kept in float32 so that the ring accumulation is stable.
+ *   - "Context parallelism", section "Ulysses Attention": an all-to-all regroups the
+ *     data so that each GPU holds all tokens of a subset of heads, and a second one
+ *     regroups the results by token.
+ *
+ * Conventions shared by every entry point:
+ *   - Layout "BSHD": [B][S][H][D] row-major, D fastest, densely packed.
+ *   - LSE layout: float32 [B][H][Sq], natural logarithm.
+ *   - Every pointer argument except chunk_bounds/bounds_out is a DEVICE pointer on
+ *     the current CUDA device, owned by the caller; the library allocates no device
+ *     memory and keeps no per-call state.  Device pointers must be 16-byte aligned.
+ *   - stream: a cudaStream_t passed as void*; NULL means the legacy default stream.
+ *     All calls are asynchronous on that stream; inputs must stay alive until the
+ *     stream has executed the call.
+ *   - Arguments are checked on the host before anything is launched; a bad argument
+ *     returns an error status and launches nothing.  No call aborts or throws.
+ *   - Device-side failures (a bounded wait that ran out) are recorded in a device
+ *     status word read by cp_last_device_status().
+ *   - Inputs must be finite; NaN/Inf inputs are outside the contract (not checked).
+ *   - Calls on the same stream are ordered; the library keeps no global state that
+ *     two streams could race on, except the device status word.
+ */
+#ifndef CPATTN_H
+#define CPATTN_H
+
+#include <stddef.h>
+
+/* Entry points are the library's only exported symbols (it is built with hidden visibility). */
+#if defined(__GNUC__)
+#define CP_API __attribute__((visibility("default")))
+#else
+#define CP_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  CP_OK = 0,
+  CP_ERR_INVALID_ARG = -1,   /* null pointer, negative size, bad chunk bounds, small workspace, bad scale */
+  CP_ERR_UNSUPPORTED = -2,   /* head_dim other than 64/128, too many chunks, size beyond 32-bit indexing */
+  CP_ERR_NOT_DIVISIBLE = -3, /* S or H not divisible by the Ulysses degree; uneven split without "anything" */
+  CP_ERR_MISALIGNED = -4,    /* a device pointer not 16-byte aligned (TMA and vector access need it) */
+  CP_ERR_CUDA = -5,          /* a CUDA runtime/driver call failed (no device, launch failure, ...) */
+  CP_ERR_TIMEOUT = -6        /* a device-side bounded wait ran out; the kernel stopped and returned */
+} cp_status;
+
+typedef enum { CP_BF16 = 0, CP_F32 = 1 } cp_dtype;
+
+/* Largest number of K/V blocks a ring simulation or a merge accepts. */
+#define CP_MAX_CHUNKS 64
+
+/*
+ * cp_attn_fwd - non-causal attention over one K/V block, returning its LSE.
+ *
+ * Source: "Attention backends", "Available backends" (scaled_dot_product_attention);
+ * "Parallelism", ContextParallelConfig.convert_to_fp32 (fp32 output + LSE per block).
+ *   S_ij = scale * q_i . k_j;  O_i = sum_j softmax_j(S_ij) v_j;  lse_i = ln sum_j exp(S_ij)
+ *
+ * q:   bf16 [B][Sq][H][D];  k, v: bf16 [B][Skv][H][D]  (device, read only)
+ * out: [B][Sq][H][D], bf16 (out_dtype CP_BF16) or fp32 (CP_F32)  (device, written)
+ * lse: fp32 [B][H][Sq] natural log (device, written), or NULL if not wanted
+ * D must be 64 or 128.  scale must be finite and > 0 (1/sqrt(D) is SDPA's default).
+ * B, H or Sq equal to 0: nothing to do, CP_OK.  Skv == 0: out = 0, lse = -inf.
+ * Computation: bf16 tensor-core products with fp32 accumulation; softmax in fp32;
+ * probabilities rounded to bf16 for the P.V product; output rounded once at the end.
+ */
+CP_API cp_status cp_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+                      int B, int H, int Sq, int Skv, int D, float scale,
+                      cp_dtype out_dtype, void* stream);
+
+/*
+ * cp_attn_fwd_blocks - attention of q over every K/V block, without the merge.
+ *
+ * Source: "Context parallelism", "Ring Attention" / "Ring Anything Attention" (each
+ * GPU attends its queries to one K/V block per ring step) and convert_to_fp32 (each
+ * block's output and LSE in float32).  Block r holds K/V rows
+ * [chunk_bounds[r], chunk_bounds[r+1]); all blocks run in one launch.
+ *
+ * chunk_bounds: HOST int[n_chunks+1], 0 = c_0 <= ... <= c_n = Skv (empty blocks allowed)
+ * partials: fp32 [n_chunks][B][Sq][H][D], lses: fp32 [n_chunks][B][H][Sq] (device, written):
+ *           exactly the inputs cp_attn_merge expects.  An empty block gives 0 and -inf.
+ * Other arguments and rules as cp_attn_fwd; 1 <= n_chunks <= CP_MAX_CHUNKS.
+ */
+CP_API cp_status cp_attn_fwd_blocks(const void* q, const void* k, const void* v, const int* chunk_bounds,
+                             int n_chunks, float* partials, float* lses, int B, int H, int Sq, int Skv,
+                             int D, float scale, void* stream);
+
+/*
+ * cp_attn_merge - combine per-block attention results through their LSEs.
+ *
+ * Source: "Context parallelism", "Ring Attention" (results accumulate over K/V
+ * blocks) and ContextParallelConfig.convert_to_fp32.  The pages print no formula;
+ * the standard log-sum-exp merge is used:
+ *   L = M + ln sum_i exp(lse_i - M),  M = max_i lse_i;   O = sum_i exp(lse_i - L) O_i
+ * A block with lse_i = -inf (no keys) has weight 0; if all are -inf, O = 0, L = -inf.
+ *
+ * partials: fp32 [n_chunks][B][Sq][H][D];  lses: fp32 [n_chunks][B][H][Sq]
+ * out: [B][Sq][H][D] in out_dtype;  out_lse: fp32 [B][H][Sq] or NULL
+ * 1 <= n_chunks <= CP_MAX_CHUNKS; D must be 64 or 128.  out may not alias partials.
+ */
+CP_API cp_status cp_attn_merge(const float* partials, const float* lses, int n_chunks, void* out,
+                        float* out_lse, int B, int H, int Sq, int D, cp_dtype out_dtype,
+                        void* stream);
+
+/* Bytes of device workspace cp_ring_sim needs: fp32 partials and LSEs of every block
+ * (n_chunks * B*H*Sq*(D+1) * 4, each part rounded up to 256 B).  0 when n_chunks == 1. */
+CP_API size_t cp_ring_sim_workspace_size(int n_chunks, int B, int H, int Sq, int D);
+
+/*
+ * cp_ring_sim - ring / ring-anything attention simulated on one GPU.
+ *
+ * Source: "Context parallelism", "Ring Attention" and "Ring Anything Attention".
+ * Block r holds K/V rows [chunk_bounds[r], chunk_bounds[r+1]); blocks are attended
+ * in ring order r = 0..n-1, each giving an fp32 partial and LSE in the workspace,
+ * then the partials are merged: cp_attn_fwd_blocks followed by cp_attn_merge.  Padded rows of ring-anything are
+ * cut away before attention on the pages, so blocks are simply their true rows.
+ *
+ * chunk_bounds: HOST int array of n_chunks+1 entries, 0 = c_0 <= c_1 <= ... <= c_n = Skv
+ *               (empty blocks allowed).  Read during the call only.
+ * workspace:    device buffer of at least cp_ring_sim_workspace_size(...) bytes,
+ *               owned by the caller; contents on return are the per-block partials.
+ * Other arguments as cp_attn_fwd.  n_chunks == 1 is plain cp_attn_fwd.
+ */
+CP_API cp_status cp_ring_sim(const void* q, const void* k, const void* v, const int* chunk_bounds,
+                      int n_chunks, void* out, float* out_lse, int B, int H, int Sq, int Skv,
+                      int D, float scale, cp_dtype out_dtype, void* workspace, size_t ws_bytes,
+                      void* stream);
+
+/*
+ * cp_ulysses_permute - the Ulysses all-to-all, simulated as one local copy.
+ *
+ * Source: "Context parallelism", "Ulysses Attention" and the variants table
+ * (sequence length and head count must be divisible by ulysses_degree).
+ * direction 0 (first exchange, sequence-sharded -> head-sharded):
+ *   src [P][B][S/P][H][D]  ->  dst [P][B][S][H/P][D]
+ *   dst[p][b][s][j][:] = src[s / (S/P)][b][s % (S/P)][p*(H/P) + j][:]
+ * direction 1: the exact inverse (second exchange, head-sharded -> sequence-sharded).
+ * P = degree >= 1.  elem_bytes: 2 (bf16/fp16) or 4 (fp32).  Bit-exact copy.
+ * S % P != 0 or H % P != 0: CP_ERR_NOT_DIVISIBLE.  src and dst may not overlap.
+ */
+CP_API cp_status cp_ulysses_permute(const void* src, void* dst, int degree, int B, int S, int H, int D,
+                             int direction, int elem_bytes, void* stream);
+
+/*
+ * cp_ring_bounds - host-only helper: block bounds for a ring of n over S rows.
+ *
+ * Source: "Context parallelism", variants table: Ring Attention needs S divisible by
+ * ring_degree; "Ring Anything Attention" accepts any S.  anything == 0: even split,
+ * CP_ERR_NOT_DIVISIBLE if S % n != 0.  anything != 0: the first S % n blocks get
+ * ceil(S/n) rows, the rest floor(S/n) (the pages do not say how ring-anything splits;
+ * this is the plainest reading).  bounds_out: HOST int[n+1].  No CUDA call.
+ */
+CP_API cp_status cp_ring_bounds(int S, int n, int anything, int* bounds_out);
+
+/* Wait for `stream`, then return and clear the device status word: CP_OK, or
+ * CP_ERR_TIMEOUT if a kernel's bounded wait ran out since the last call.  Returns
+ * CP_ERR_CUDA if the stream reported an error. */
+CP_API cp_status cp_last_device_status(void* stream);
+
+/* Static string naming a status code. */
+CP_API const char* cp_status_string(cp_status s);
+
+/* Library ABI version (major*100 + minor). */
+CP_API int cp_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CPATTN_H */

@@ -1,0 +1,150 @@
+"""The C ABI on the host: the library loads, exports every declared entry point and
+rejects bad arguments before launching anything (no GPU needed)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from context_attention_dit_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "cpattn.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(cp_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_loads_and_exports_header(lib):
+    names = declared_functions()
+    assert "cp_attn_fwd" in names and "cp_ulysses_permute" in names
+    for name in names:
+        assert hasattr(lib, name), f"libcpattn.so does not export {name}"
+    assert set(binding.EXPORTS) <= set(names)
+
+
+def test_exported_symbols_in_dynamic_table():
+    import subprocess
+
+    out = subprocess.run(["nm", "-D", "--defined-only", binding.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\b(cp_[a-z0-9_]+)\b", out))
+    assert set(declared_functions()) <= exported
+
+
+def test_version_and_strings(lib):
+    assert lib.cp_version() == 100
+    for code in (0, -1, -2, -3, -4, -5, -6):
+        assert binding.status_string(code).startswith("CP_")
+
+
+I = binding
+
+
+@pytest.mark.parametrize(
+    "args,want",
+    [
+        # q, k, v, out, lse, B, H, Sq, Skv, D, scale, dtype
+        ((None, None, None, None, None, 1, 2, 16, 16, 96, 0.1, 0), I.CP_ERR_UNSUPPORTED),   # head_dim
+        ((None, None, None, None, None, -1, 2, 16, 16, 64, 0.1, 0), I.CP_ERR_INVALID_ARG),  # negative size
+        ((None, None, None, None, None, 1, 2, 16, 16, 64, 0.0, 0), I.CP_ERR_INVALID_ARG),   # scale <= 0
+        ((None, None, None, None, None, 1, 2, 16, 16, 64, float("nan"), 0), I.CP_ERR_INVALID_ARG),
+        ((None, None, None, None, None, 1, 2, 16, 16, 64, 0.1, 7), I.CP_ERR_INVALID_ARG),   # dtype code
+        ((None, None, None, None, None, 1, 2, 16, 16, 64, 0.1, 0), I.CP_ERR_INVALID_ARG),   # null pointers
+        ((16, 32, 48, 8, None, 1, 2, 16, 16, 64, 0.1, 0), I.CP_ERR_MISALIGNED),            # out not 16B aligned
+        ((None, None, None, None, None, 0, 2, 16, 16, 64, 0.1, 0), I.CP_OK),                # empty batch: no-op
+    ],
+)
+def test_attn_fwd_rejects_before_launch(lib, args, want):
+    *ptrs, B, H, Sq, Skv, D, scale, dt = args
+    st = lib.cp_attn_fwd(*[ctypes.c_void_p(p) if p else None for p in ptrs], B, H, Sq, Skv, D, scale, dt, None)
+    assert st == want
+
+
+def test_merge_rejects(lib):
+    assert lib.cp_attn_merge(None, None, 0, None, None, 1, 1, 1, 64, 0, None) == I.CP_ERR_INVALID_ARG
+    assert lib.cp_attn_merge(None, None, 65, None, None, 1, 1, 1, 64, 0, None) == I.CP_ERR_UNSUPPORTED
+    assert lib.cp_attn_merge(None, None, 2, None, None, 1, 1, 1, 32, 0, None) == I.CP_ERR_UNSUPPORTED
+    assert lib.cp_attn_merge(None, None, 2, None, None, 1, 1, 1, 64, 0, None) == I.CP_ERR_INVALID_ARG
+    assert lib.cp_attn_merge(ctypes.c_void_p(32), ctypes.c_void_p(64), 2, ctypes.c_void_p(4), None, 1, 1, 1, 64, 0,
+                             None) == I.CP_ERR_MISALIGNED
+
+
+def _bounds(*c):
+    return (ctypes.c_int * len(c))(*c)
+
+
+@pytest.mark.parametrize(
+    "bounds,n,skv,want",
+    [
+        ((0, 8, 16), 2, 16, I.CP_ERR_INVALID_ARG),     # null q etc. after bounds pass
+        ((1, 8, 16), 2, 16, I.CP_ERR_INVALID_ARG),     # does not start at 0
+        ((0, 8, 15), 2, 16, I.CP_ERR_INVALID_ARG),     # does not end at Skv
+        ((0, 9, 8, 16), 3, 16, I.CP_ERR_INVALID_ARG),  # not monotonic
+        ((0, 16), 0, 16, I.CP_ERR_INVALID_ARG),        # no blocks
+    ],
+)
+def test_ring_sim_rejects_bad_bounds(lib, bounds, n, skv, want):
+    st = lib.cp_ring_sim(None, None, None, _bounds(*bounds), n, None, None, 1, 2, 16, skv, 64, 0.1, 0, None, 0, None)
+    assert st == want
+
+
+def test_ring_sim_rejects_small_workspace(lib):
+    # pointers are fake but aligned; the workspace check comes before any CUDA call
+    p = ctypes.c_void_p(1 << 20)
+    st = lib.cp_ring_sim(p, p, p, _bounds(0, 8, 16), 2, p, None, 1, 2, 16, 16, 64, 0.1, 0, p, 100, None)
+    assert st == I.CP_ERR_INVALID_ARG
+
+
+def test_workspace_size(lib):
+    assert binding.ring_workspace_size(1, 1, 24, 4608, 128) == 0
+    n, B, H, S, D = 8, 1, 24, 4608, 128
+    want = n * B * H * S * D * 4 + n * B * H * S * 4
+    assert binding.ring_workspace_size(n, B, H, S, D) == want
+
+
+def test_ring_bounds():
+    assert binding.ring_bounds(4608, 8) == [576 * i for i in range(9)]
+    assert binding.ring_bounds(4173, 3, anything=True) == [0, 1391, 2782, 4173]
+    assert binding.ring_bounds(4481, 4, anything=True) == [0, 1121, 2241, 3361, 4481]
+    with pytest.raises(binding.CpError) as e:
+        binding.ring_bounds(4481, 4)
+    assert e.value.status == I.CP_ERR_NOT_DIVISIBLE
+
+
+def test_permute_rejects(lib):
+    assert lib.cp_ulysses_permute(None, None, 0, 1, 8, 8, 64, 0, 2, None) == I.CP_ERR_INVALID_ARG
+    assert lib.cp_ulysses_permute(None, None, 2, 1, 8, 8, 64, 2, 2, None) == I.CP_ERR_INVALID_ARG
+    assert lib.cp_ulysses_permute(None, None, 2, 1, 8, 8, 64, 0, 3, None) == I.CP_ERR_UNSUPPORTED
+    assert lib.cp_ulysses_permute(None, None, 3, 1, 8, 9, 64, 0, 2, None) == I.CP_ERR_NOT_DIVISIBLE
+    assert lib.cp_ulysses_permute(None, None, 3, 1, 9, 8, 64, 0, 2, None) == I.CP_ERR_NOT_DIVISIBLE
+    p = ctypes.c_void_p(1 << 20)
+    assert lib.cp_ulysses_permute(p, p, 2, 1, 8, 8, 64, 0, 2, None) == I.CP_ERR_INVALID_ARG  # overlap
+
+
+def _golden_rows():
+    rows = []
+    for line in open(os.path.join(ROOT, "tests", "golden", "divisibility_flux.txt")):
+        line = line.split("#", 1)[0].strip()
+        if line:
+            res, tok, heads, variant, deg, want = line.split()
+            rows.append((int(res), int(tok), int(heads), variant, int(deg), want))
+    return rows
+
+
+@pytest.mark.parametrize("row", _golden_rows(), ids=lambda r: f"{r[0]}-{r[3]}-{r[4]}")
+def test_pages_divisibility_rules(lib, row):
+    res, tokens, heads, variant, degree, want = row
+    if variant in ("ring", "ring_anything"):
+        out = (ctypes.c_int * (degree + 1))()
+        st = lib.cp_ring_bounds(tokens, degree, 1 if variant == "ring_anything" else 0, out)
+        assert (st == I.CP_OK) == (want == "ok")
+        if st == I.CP_OK:
+            sizes = [out[i + 1] - out[i] for i in range(degree)]
+            assert sum(sizes) == tokens and max(sizes) - min(sizes) <= 1
+    else:  # ulysses: null pointers pass the divisibility check and stop at the pointer check
+        st = lib.cp_ulysses_permute(None, None, degree, 1, tokens, heads, 128, 0, 2, None)
+        assert st == (I.CP_ERR_INVALID_ARG if want == "ok" else I.CP_ERR_NOT_DIVISIBLE)

@@ -1,0 +1,132 @@
+"""cp_attn_fwd (tcgen05 attention kernel) against the fp64 oracle, through the C ABI."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from context_attention_dit_b200 import binding
+from tests.gpu_util import assert_attn_close, cuda, qkv, workload_inputs, workload_oracle
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [
+    # B, H, Sq, Skv, D      (several tiles, ragged tails, single rows)
+    (1, 8, 10, 10, 64),      # the pages' dispatcher example shape (1, 10, 8, 64)
+    (1, 2, 256, 256, 64),
+    (2, 3, 129, 300, 128),
+    (1, 2, 1, 1, 128),
+    (1, 1, 127, 129, 64),
+    (1, 2, 384, 1000, 128),
+    (2, 2, 200, 77, 128),
+    (1, 4, 1391, 1391, 128),
+    (3, 1, 64, 4173, 64),
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32], ids=["bf16", "fp32"])
+def test_attn_matches_oracle(shape, out_dtype):
+    B, H, Sq, Skv, D = shape
+    q, k, v = qkv(B, H, Sq, Skv, D, seed=7)
+    scale = 1.0 / math.sqrt(D)
+    o_ref, lse_ref = oracle.attention(q, k, v, scale)
+    o, lse = binding.attn_fwd(*cuda(q, k, v), scale=scale, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    assert binding.last_device_status() == 0
+    assert_attn_close(o, lse, o_ref, lse_ref, f"attn {shape}")
+
+
+def test_attn_no_keys():
+    q, k, v = qkv(1, 2, 130, 0, 128)
+    o, lse = binding.attn_fwd(*cuda(q, k, v))
+    torch.cuda.synchronize()
+    assert not o.float().abs().sum().item()
+    assert torch.isneginf(lse).all()
+
+
+def test_attn_nonstandard_scale_and_large_logits():
+    """scale 0.9 on N(0, 2^2) inputs: logits of |s| ~ 100 exercise the lazy rescaling of O."""
+    B, H, Sq, Skv, D = 1, 2, 256, 1024, 128
+    g = torch.Generator().manual_seed(3)
+    q = (torch.randn(B, Sq, H, D, generator=g) * 2).bfloat16()
+    k = (torch.randn(B, Skv, H, D, generator=g) * 2).bfloat16()
+    v = torch.randn(B, Skv, H, D, generator=g).bfloat16()
+    o_ref, lse_ref = oracle.attention(q, k, v, 0.09)
+    o, lse = binding.attn_fwd(*cuda(q, k, v), scale=0.09, out_dtype=torch.float32)
+    assert_attn_close(o, lse, o_ref, lse_ref, "large logits")
+
+
+def test_identical_keys_give_mean_of_v():
+    """Closed form on the GPU: all keys equal -> every output row is mean_j v_j."""
+    B, H, Sq, Skv, D = 1, 2, 200, 600, 128
+    q, _, v = qkv(B, H, Sq, Skv, D, seed=11)
+    k = qkv(B, H, 1, 1, D, seed=12)[1].expand(B, Skv, H, D).contiguous()
+    o, lse = binding.attn_fwd(*cuda(q, k, v), out_dtype=torch.float32)
+    want = v.float().mean(dim=1, keepdim=True).expand_as(o.cpu())
+    assert (o.cpu() - want).abs().max().item() < 5e-3
+    logit = (q.float() * k[:, :1].float()).sum(-1).permute(0, 2, 1) / math.sqrt(D)
+    assert (lse.cpu() - (math.log(Skv) + logit)).abs().max().item() < 1e-3
+
+
+def test_dominant_logit_selects_its_row():
+    """q_i = 8*k_{j*}: one logit dominates by ~8*sqrt(D)/... so o_i is v_{j*} to bf16 precision."""
+    B, H, Sq, Skv, D = 1, 1, 128, 512, 128
+    _, k, v = qkv(B, H, Sq, Skv, D, seed=13, rms=True)
+    idx = torch.arange(Sq) * 3 % Skv
+    q = (k[:, idx].float() * 8).bfloat16()
+    o, _ = binding.attn_fwd(*cuda(q, k, v), out_dtype=torch.float32)
+    assert (o.cpu() - v[:, idx].float()).abs().max().item() < 2e-2
+
+
+def test_flux_full_attention_all_elements():
+    """FLUX.1-dev 1024^2 joint attention (B1 H24 S4608 D128, QK-normed): every element vs fp64."""
+    w, (q, k, v) = workload_inputs("flux_1024_ring1")
+    o_ref, lse_ref = workload_oracle("flux_1024_ring1")
+    o, lse = binding.attn_fwd(*cuda(q, k, v), scale=w.scale)
+    stats = assert_attn_close(o, lse, o_ref, lse_ref, "flux ring-1")
+    print("flux ring-1 max/mean/relL2", stats)
+
+
+def test_deterministic_bitwise():
+    q, k, v = cuda(*qkv(1, 4, 700, 900, 128, seed=21))
+    outs = [binding.attn_fwd(q, k, v, out_dtype=torch.float32) for _ in range(3)]
+    for o, l in outs[1:]:
+        assert torch.equal(o, outs[0][0]) and torch.equal(l, outs[0][1])
+
+
+def test_guard_regions_and_full_write():
+    """Outputs pre-filled with NaN are fully written; sentinel guard bytes on both sides stay intact."""
+    B, H, Sq, Skv, D = 1, 3, 333, 257, 128
+    q, k, v = cuda(*qkv(B, H, Sq, Skv, D, seed=5))
+    guard = 4096
+    n_o, n_l = B * Sq * H * D, B * H * Sq
+    obuf = torch.full((n_o + 2 * guard,), float("nan"), dtype=torch.float32, device="cuda")
+    lbuf = torch.full((n_l + 2 * guard,), float("nan"), dtype=torch.float32, device="cuda")
+    obuf[:guard] = 12345.0
+    obuf[-guard:] = 12345.0
+    lbuf[:guard] = -777.0
+    lbuf[-guard:] = -777.0
+    o = obuf[guard:guard + n_o].view(B, Sq, H, D)
+    lse = lbuf[guard:guard + n_l].view(B, H, Sq)
+    binding.attn_fwd(q, k, v, out_dtype=torch.float32, out=o, lse=lse)
+    torch.cuda.synchronize()
+    assert torch.isfinite(o).all() and torch.isfinite(lse).all()
+    assert (obuf[:guard] == 12345.0).all() and (obuf[-guard:] == 12345.0).all()
+    assert (lbuf[:guard] == -777.0).all() and (lbuf[-guard:] == -777.0).all()
+
+
+def test_binding_checks_mirror_dispatcher():
+    q, k, v = cuda(*qkv(1, 2, 16, 16, 64))
+    with pytest.raises(ValueError):
+        binding.attn_fwd(q.float(), k, v)               # dtype
+    with pytest.raises(ValueError):
+        binding.attn_fwd(q, k[:, :, :1].contiguous(), v)  # shape
+    with pytest.raises(ValueError):
+        binding.attn_fwd(q.cpu(), k, v)                 # device
+    q96, k96, v96 = cuda(*qkv(1, 2, 16, 16, 96))
+    with pytest.raises(binding.CpError) as e:
+        binding.attn_fwd(q96, k96, v96)
+    assert e.value.status == binding.CP_ERR_UNSUPPORTED
