@@ -61,14 +61,15 @@ def load() -> ctypes.CDLL:
     lib.cp_ring_sim_workspace_size.argtypes = [i, i, i, i, i]
     lib.cp_ring_sim_workspace_size.restype = sz
     lib.cp_ring_sim.argtypes = [vp, vp, vp, ip, i, vp, vp, i, i, i, i, i, f, i, vp, sz, vp]
+    lib.cp_ring_sim_static.argtypes = [vp, vp, vp, ip, i, vp, vp, i, i, i, i, i, f, i, vp]
     lib.cp_ulysses_permute.argtypes = [vp, vp, i, i, i, i, i, i, i, vp]
     lib.cp_ring_bounds.argtypes = [i, i, i, ip]
     lib.cp_last_device_status.argtypes = [vp]
     lib.cp_status_string.argtypes = [i]
     lib.cp_status_string.restype = ctypes.c_char_p
     lib.cp_version.argtypes = []
-    for name in ("cp_attn_fwd", "cp_attn_fwd_blocks", "cp_attn_merge", "cp_ring_sim", "cp_ulysses_permute", "cp_ring_bounds",
-                 "cp_last_device_status"):
+    for name in ("cp_attn_fwd", "cp_attn_fwd_blocks", "cp_attn_merge", "cp_ring_sim", "cp_ring_sim_static", "cp_ulysses_permute",
+                 "cp_ring_bounds", "cp_last_device_status"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -203,6 +204,40 @@ def ring_sim(q, k, v, chunk_bounds: Sequence[int], scale: Optional[float] = None
                             code, _ptr(workspace), ws_bytes, ctypes.c_void_p(_stream(q)))
     _check(st, "cp_ring_sim")
     return out, out_lse, workspace
+
+
+STATIC_SCRATCH_BYTES = 32 << 20
+
+
+def ring_sim_static(q, k, v, chunk_bounds: Sequence[int], scale: Optional[float] = None, out_dtype=torch.bfloat16,
+                    out=None, out_lse=None):
+    """:func:`ring_sim` without a workspace, for callers that cannot allocate device memory.
+
+    The per-block partials live in the library's static 32 MiB device array, so the
+    library call allocates nothing (``out``/``out_lse`` are allocated here only when not
+    given; pass them to allocate nothing at all).  Problems whose partials exceed the
+    array raise ``CpError`` (``CP_ERR_UNSUPPORTED``).  Calls that overlap on the GPU share
+    the array and race.  Make the first call on a device before any stream capture.
+    """
+    B, Sq, Skv, H, D = _check_qkv(q, k, v)
+    code = _out_code(out_dtype)
+    scale = float(D ** -0.5 if scale is None else scale)
+    n = len(chunk_bounds) - 1
+    if n < 1:
+        raise ValueError("chunk_bounds needs at least two entries")
+    need = ring_workspace_size(n, B, H, Sq, D)
+    if need > STATIC_SCRATCH_BYTES:
+        raise CpError(CP_ERR_UNSUPPORTED, f"cp_ring_sim_static (needs {need} bytes of scratch, the static array "
+                                          f"holds {STATIC_SCRATCH_BYTES})")
+    bounds = (ctypes.c_int * (n + 1))(*[int(c) for c in chunk_bounds])
+    if out is None:
+        out = torch.empty((B, Sq, H, D), dtype=out_dtype, device=q.device)
+    if out_lse is None:
+        out_lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
+    st = load().cp_ring_sim_static(_ptr(q), _ptr(k), _ptr(v), bounds, n, _ptr(out), _ptr(out_lse), B, H, Sq, Skv, D,
+                                   scale, code, ctypes.c_void_p(_stream(q)))
+    _check(st, "cp_ring_sim_static")
+    return out, out_lse
 
 
 def ring_workspace_views(workspace, n: int, B: int, H: int, Sq: int, D: int):

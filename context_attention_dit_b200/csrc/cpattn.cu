@@ -277,6 +277,52 @@ cp_status cp_ring_sim(const void* q, const void* k, const void* v, const int* ch
   return launch_merge(partials, lses, n_chunks, out, out_lse, B, H, Sq, D, out_dtype, s);
 }
 
+}  // extern "C"
+
+// Static scratch of cp_ring_sim_static: fp32 partials and LSEs of every K/V block, for
+// callers that cannot allocate.  Host code only ever sees a stand-in for this symbol,
+// so its device address is looked up per device (with that device current) and passed
+// to the kernels as an ordinary pointer.
+static __device__ __align__(256) unsigned char g_static_scratch[CP_STATIC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_scratch_mutex;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+cp_status static_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CP_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return CP_ERR_CUDA;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return CP_OK;
+}
+}  // namespace
+
+extern "C" {
+
+cp_status cp_ring_sim_static(const void* q, const void* k, const void* v, const int* chunk_bounds, int n_chunks,
+                             void* out, float* out_lse, int B, int H, int Sq, int Skv, int D, float scale,
+                             cp_dtype out_dtype, void* stream) {
+  cp_status st = check_bounds(chunk_bounds, n_chunks, Skv);
+  if (st != CP_OK) return st;
+  st = check_attn_args(q, k, v, out, out_lse, B, H, Sq, Skv, D, scale, out_dtype);
+  if (st != CP_OK || B == 0 || H == 0 || Sq == 0) return st;
+  const size_t need = cp_ring_sim_workspace_size(n_chunks, B, H, Sq, D);
+  if (need > CP_STATIC_SCRATCH_BYTES) return CP_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  if (need > 0) {
+    st = static_scratch(&scratch);
+    if (st != CP_OK) return st;
+  }
+  return cp_ring_sim(q, k, v, chunk_bounds, n_chunks, out, out_lse, B, H, Sq, Skv, D, scale, out_dtype, scratch,
+                     need, stream);
+}
+
 cp_status cp_ulysses_permute(const void* src, void* dst, int degree, int B, int S, int H, int D, int direction,
                              int elem_bytes, void* stream) {
   if (degree < 1 || B < 0 || S < 0 || H < 0 || D < 0) return CP_ERR_INVALID_ARG;

@@ -139,6 +139,36 @@ CP_API cp_status cp_ring_sim(const void* q, const void* k, const void* v, const 
                       int D, float scale, cp_dtype out_dtype, void* workspace, size_t ws_bytes,
                       void* stream);
 
+/* Size in bytes of the library's static device scratch used by cp_ring_sim_static. */
+#define CP_STATIC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * cp_ring_sim_static - cp_ring_sim for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart to this call; it exists for users of this library
+ * whose code may not call cudaMalloc (or any allocator) when they attend: code
+ * running inside another framework's memory pool, during CUDA stream capture,
+ * or in a real-time loop that must not allocate.  It computes exactly what
+ * cp_ring_sim computes, with the same arguments minus workspace/ws_bytes: the
+ * per-block fp32 partials and LSEs live in one file-scope device array of
+ * CP_STATIC_SCRATCH_BYTES (32 MiB) that every GPU which loads the library keeps
+ * until the process exits.  The call allocates nothing.
+ *
+ * - Sizes: if cp_ring_sim_workspace_size(n_chunks, B, H, Sq, D) exceeds
+ *   CP_STATIC_SCRATCH_BYTES the call returns CP_ERR_UNSUPPORTED and launches nothing.
+ * - Set-up: the first call on a device looks up the array's device address with
+ *   that device current (cudaGetSymbolAddress); make that first call before any
+ *   stream capture.  A failed look-up returns CP_ERR_CUDA.
+ * - Sharing: every call on every stream of a device uses the same array.  Calls
+ *   that overlap on the GPU (different streams, no ordering) race and corrupt each
+ *   other's results; order them on one stream or with events.  The array keeps the
+ *   last call's partials; nothing needs clearing, because every partial and LSE
+ *   entry a call reads is written by that call first.
+ */
+CP_API cp_status cp_ring_sim_static(const void* q, const void* k, const void* v, const int* chunk_bounds,
+                             int n_chunks, void* out, float* out_lse, int B, int H, int Sq, int Skv,
+                             int D, float scale, cp_dtype out_dtype, void* stream);
+
 /*
  * cp_ulysses_permute - the Ulysses all-to-all, simulated as one local copy.
  *
