@@ -7,24 +7,32 @@
 // per-block fp32 output + LSE follow ContextParallelConfig.convert_to_fp32 on the
 // "Parallelism" API page, so that ring blocks can be merged afterwards).
 //
-// Design (one CTA per SM, persistent over work items (b, h, c, q-tile)):
-//   warp 0      TMA producer: Q tile (128 rows x D) once per item, then K and V tiles
-//               (128 keys x D) through a ring of kStages shared-memory stages.
-//   warp 1      allocates TMEM; one elected thread issues every tcgen05.mma:
-//               S = Q K^T (SS form, K-major operands) into a double-buffered S in TMEM,
-//               O += P V (TS form: P read from TMEM, V MN-major from shared memory).
-//   warps 2..5  softmax warpgroup: thread t of warp w owns query row 32*(w%4)+t, which
-//               is TMEM lane 32*(w%4)+t.  It loads its S row (fp32), masks keys past the
-//               block end, updates the running max m / sum l (base-2 domain), writes
-//               P = 2^(S*scale*log2e - m) as bf16 pairs over the first 64 columns of
-//               the same S buffer, and after the last tile writes O/l and the LSE.
-// The running max is updated lazily: O (in TMEM) is rescaled only when a row's max
-// grows by more than 8 (a factor 256); otherwise the stale max stays, which is exact
-// because O and l share it and 2^8 cannot overflow fp32 or bf16.
-// TMEM columns: S buffers at [0,128) and [128,256), O at [256, 256+D).
-// Every mbarrier wait is bounded (see ptx_sm100.cuh); on a timeout every role leaves
-// its loop, in-flight TMA loads and MMAs are drained, TMEM is freed and the kernel
-// returns with CP_ERR_TIMEOUT recorded in the device status word.
+// Design (one CTA per SM, persistent over work units (b, h, pair of 128-row Q tiles);
+// each unit walks every K/V block and, inside a block, its 128-key tiles):
+//   warps 0-3   softmax warpgroup 0, Q tile 0 of the pair; thread t of warp w owns
+//   warps 4-7   softmax warpgroup 1, Q tile 1; its query row 32*(w%4)+t = TMEM lane.
+//               Per K/V tile: load the S row from TMEM, mask keys past the block end,
+//               update the running max m and sum l (base 2), write P = 2^(S*scale*log2e
+//               - m) as bf16 pairs into the first columns of the same S buffer.  After
+//               a block's last tile: write O/l (fp32 partial or final bf16/fp32) and lse.
+//   warp 8      TMA producer: both Q tiles once per unit; K and V tiles (128 keys x D)
+//               through two 2-stage rings.  Warps 8-11 form the control warpgroup, which
+//               hands registers to the softmax warpgroups (setmaxnreg 88 / 208).
+//   warp 9      TMEM owner (512 columns) and MMA issuer (one thread), in the order
+//               QK0(t) QK1(t) | PV0(t) QK0(t+1) PV1(t) QK1(t+1) | ...
+//               S_w = Q_w K^T: SS form, both operands K-major and 128B-swizzled;
+//               O_w += P_w V: TS form, P_w read from TMEM, V MN-major in shared memory.
+//               Because QK_w(t+1) is issued after PV_w(t), the commit that signals "S_w
+//               full" also certifies that O_w holds every earlier P.V product.
+// TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [384,384+D).
+// A tile whose block has at most 64 keys left runs N = 64 (QK) and K = 64 (PV) MMAs and
+// a 64-column softmax.
+// The running max is updated lazily: O_w is rescaled in TMEM only when a row's max grows
+// by more than 8 (a factor 256); otherwise the stale max stays, which is exact because O
+// and l share it and 2^8 cannot overflow fp32 or bf16.
+// Every mbarrier wait is bounded (see ptx_sm100.cuh); on a timeout every role leaves its
+// loop, in-flight TMA loads and MMAs are drained, TMEM is freed and the kernel returns
+// with CP_ERR_TIMEOUT recorded in the device status word.
 #pragma once
 
 #include <cuda.h>
@@ -33,10 +41,17 @@
 
 namespace cpattn {
 
-constexpr int kBM = 128;          // query rows per tile (TMEM lanes)
-constexpr int kBN = 128;          // keys per K/V tile
-constexpr int kStages = 2;        // K/V shared-memory stages
-constexpr int kAttnThreads = 192; // 6 warps
+constexpr int kBM = 128;           // query rows per Q tile (TMEM lanes)
+constexpr int kQTiles = 2;         // Q tiles per work unit, one softmax warpgroup each
+constexpr int kBN = 128;           // keys per K/V tile
+constexpr int kStages = 2;         // stages of each of the K and V rings
+constexpr int kAttnThreads = 384;  // 12 warps: two softmax warpgroups + a control warpgroup
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+// Registers per thread after the split (launch: 168 = 65536 / 384 rounded down to 8).
+// 256 * 208 + 128 * 88 = 384 * 168.
+constexpr int kSoftmaxRegs = 208;
+constexpr int kControlRegs = 88;
 constexpr int kTmemCols = 512;
 constexpr int kMaxChunks = 64;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -44,13 +59,14 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 struct AttnParams {
   int B, H, Sq;
   int n_chunks;
-  int n_qt;                  // ceil(Sq / kBM)
-  int total_items;           // B * H * n_chunks * n_qt
+  int n_qp;                  // ceil(Sq / (kQTiles * kBM)) Q-tile pairs
+  int n_units;               // B * H * n_qp
+  int tiles_per_unit;        // sum over blocks of ceil(len / kBN)
   float scale_log2;          // scale * log2(e)
-  void* out;                 // chunk c at out + c*out_chunk_stride elements, [B][Sq][H][D]
+  void* out;                 // block c at out + c*out_chunk_stride elements, [B][Sq][H][D]
   int out_f32;               // 1: fp32 output, 0: bf16 output
   long long out_chunk_stride;
-  float* lse;                // chunk c at lse + c*lse_chunk_stride, [B][H][Sq]; may be null
+  float* lse;                // block c at lse + c*lse_chunk_stride, [B][H][Sq]; may be null
   long long lse_chunk_stride;
   int* status;               // device status word
   int bounds[kMaxChunks + 1];  // K/V row bounds of the blocks
@@ -58,32 +74,78 @@ struct AttnParams {
 
 template <int D>
 struct AttnSmem {
-  static constexpr int kHalfBytes = kBM * 64 * 2;          // 128 rows x 64 bf16 = one 128B-swizzled box
-  static constexpr int kTileBytes = kBM * D * 2;           // 128 rows x D bf16
-  static constexpr int kQ = 0;
-  static constexpr int kK = kQ + kTileBytes;
+  static constexpr int kHalfBytes = kBM * 64 * 2;  // 128 rows x 64 bf16: one 128B-swizzled box
+  static constexpr int kTileBytes = kBM * D * 2;   // 128 rows x D bf16
+  static constexpr int kQ = 0;                     // kQTiles Q tiles
+  static constexpr int kK = kQ + kQTiles * kTileBytes;
   static constexpr int kV = kK + kStages * kTileBytes;
   static constexpr int kBar = kV + kStages * kTileBytes;
-  static constexpr int kNumBars = 17;
+  static constexpr int kNumBars = 19;
   static constexpr int kUsed = kBar + kNumBars * 8 + 16;
-  // Ask for more than half an SM's shared memory so that exactly one CTA (which owns
-  // all 512 TMEM columns) is resident per SM.
+  // More than half an SM's shared memory: exactly one CTA (owning all 512 TMEM
+  // columns) is resident per SM.
   static constexpr int kRequest = (kUsed + 1024) > 120 * 1024 ? (kUsed + 1024) : 120 * 1024;
 };
 
-struct ItemCoord {
-  int b, h, c, qt;
+// Barrier indices.
+enum : int {
+  kQFull = 0, kQEmpty = 1, kKFull = 2, kKEmpty = 4, kVFull = 6, kVEmpty = 8,
+  kSFull = 10, kPReady = 12, kODone = 14, kOFree = 16, kDrain = 18
 };
 
-__device__ __forceinline__ ItemCoord decode_item(int item, const AttnParams& p) {
-  ItemCoord r;
-  r.qt = item % p.n_qt;
-  int t = item / p.n_qt;
-  r.c = t % p.n_chunks;
-  t /= p.n_chunks;
-  r.h = t % p.H;
-  r.b = t / p.H;
+struct UnitCoord {
+  int b, h, qp;
+};
+
+__device__ __forceinline__ UnitCoord decode_unit(int u, const AttnParams& p) {
+  UnitCoord r;
+  r.qp = u % p.n_qp;
+  const int bh = u / p.n_qp;
+  r.h = bh % p.H;
+  r.b = bh / p.H;
   return r;
+}
+
+// One 128-key (or shorter) tile of K/V block c.
+struct Tile {
+  int c, j;     // block, tile within the block
+  int row0;     // first K/V row
+  int valid;    // keys of the block in this tile (1..128)
+  bool first, last;
+};
+
+__device__ __forceinline__ int block_tiles(const AttnParams& p, int c) {
+  return (p.bounds[c + 1] - p.bounds[c] + kBN - 1) / kBN;
+}
+
+__device__ __forceinline__ Tile make_tile(const AttnParams& p, int c, int j) {
+  Tile t;
+  t.c = c;
+  t.j = j;
+  const int len = p.bounds[c + 1] - p.bounds[c];
+  t.row0 = p.bounds[c] + j * kBN;
+  t.valid = min(kBN, len - j * kBN);
+  t.first = (j == 0);
+  t.last = (j == (len + kBN - 1) / kBN - 1);
+  return t;
+}
+
+// First tile at or after block c (skipping empty blocks); false if none.
+__device__ __forceinline__ bool first_tile_from(const AttnParams& p, int c, Tile& t) {
+  for (; c < p.n_chunks; ++c)
+    if (block_tiles(p, c) > 0) {
+      t = make_tile(p, c, 0);
+      return true;
+    }
+  return false;
+}
+
+__device__ __forceinline__ bool next_tile(const AttnParams& p, const Tile& cur, Tile& nxt) {
+  if (!cur.last) {
+    nxt = make_tile(p, cur.c, cur.j + 1);
+    return true;
+  }
+  return first_tile_from(p, cur.c + 1, nxt);
 }
 
 // All lanes wait; the warp proceeds only if every lane saw the phase complete.
@@ -100,313 +162,345 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// ------------------------------------------------------------------------------- producer
+
 template <int D>
 __device__ __forceinline__ void attn_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
                                               const CUtensorMap* tm_v, const AttnParams& p, uint8_t* smem,
                                               uint64_t* bars, volatile int* abort_flag) {
   using L = AttnSmem<D>;
-  uint64_t* q_full = bars + 0;
-  uint64_t* q_empty = bars + 1;
-  uint64_t* k_full = bars + 2;
-  uint64_t* k_empty = bars + 4;
-  uint64_t* v_full = bars + 6;
-  uint64_t* v_empty = bars + 8;
+  if (p.tiles_per_unit == 0) return;
   uint32_t kc_k = 0, kc_v = 0;  // tiles issued into the K and V rings
-  int t_ne = 0;                 // items with at least one K/V tile
+  uint32_t n_q = 0;             // Q pairs issued
   bool ok = true;
-  for (int item = blockIdx.x; item < p.total_items && ok; item += gridDim.x) {
-    const ItemCoord ic = decode_item(item, p);
-    const int kv0 = p.bounds[ic.c];
-    const int kvlen = p.bounds[ic.c + 1] - kv0;
-    const int n_kv = (kvlen + kBN - 1) / kBN;
-    if (n_kv == 0) continue;
-    if (t_ne > 0 && !mbar_wait(q_empty, (t_ne - 1) & 1, abort_flag, p.status)) break;
-    mbar_arrive_expect_tx(q_full, L::kTileBytes);
+  for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+    const UnitCoord uc = decode_unit(u, p);
+    if (n_q > 0 && !mbar_wait(bars + kQEmpty, (n_q - 1) & 1, abort_flag, p.status)) break;
+    mbar_arrive_expect_tx(bars + kQFull, kQTiles * L::kTileBytes);
 #pragma unroll
-    for (int hf = 0; hf < D / 64; ++hf)
-      tma_load_4d(smem + L::kQ + hf * L::kHalfBytes, tm_q, q_full, hf * 64, ic.h, ic.qt * kBM, ic.b);
-    ++t_ne;
-    for (int j = 0; j < n_kv; ++j) {
-      const int row = kv0 + j * kBN;
+    for (int w = 0; w < kQTiles; ++w)
+#pragma unroll
+      for (int hf = 0; hf < D / 64; ++hf)
+        tma_load_4d(smem + L::kQ + w * L::kTileBytes + hf * L::kHalfBytes, tm_q, bars + kQFull, hf * 64, uc.h,
+                    (uc.qp * kQTiles + w) * kBM, uc.b);
+    ++n_q;
+    Tile t;
+    bool have = first_tile_from(p, 0, t);
+    while (have) {
       {
         const int st = kc_k % kStages;
-        const uint32_t u = kc_k / kStages;
-        if (u > 0 && !mbar_wait(k_empty + st, (u - 1) & 1, abort_flag, p.status)) { ok = false; break; }
-        mbar_arrive_expect_tx(k_full + st, L::kTileBytes);
+        const uint32_t use = kc_k / kStages;
+        if (use > 0 && !mbar_wait(bars + kKEmpty + st, (use - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+        mbar_arrive_expect_tx(bars + kKFull + st, L::kTileBytes);
 #pragma unroll
         for (int hf = 0; hf < D / 64; ++hf)
-          tma_load_4d(smem + L::kK + st * L::kTileBytes + hf * L::kHalfBytes, tm_k, k_full + st, hf * 64, ic.h,
-                      row, ic.b);
+          tma_load_4d(smem + L::kK + st * L::kTileBytes + hf * L::kHalfBytes, tm_k, bars + kKFull + st, hf * 64,
+                      uc.h, t.row0, uc.b);
         ++kc_k;
       }
       {
         const int st = kc_v % kStages;
-        const uint32_t u = kc_v / kStages;
-        if (u > 0 && !mbar_wait(v_empty + st, (u - 1) & 1, abort_flag, p.status)) { ok = false; break; }
-        mbar_arrive_expect_tx(v_full + st, L::kTileBytes);
+        const uint32_t use = kc_v / kStages;
+        if (use > 0 && !mbar_wait(bars + kVEmpty + st, (use - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+        mbar_arrive_expect_tx(bars + kVFull + st, L::kTileBytes);
 #pragma unroll
         for (int hf = 0; hf < D / 64; ++hf)
-          tma_load_4d(smem + L::kV + st * L::kTileBytes + hf * L::kHalfBytes, tm_v, v_full + st, hf * 64, ic.h,
-                      row, ic.b);
+          tma_load_4d(smem + L::kV + st * L::kTileBytes + hf * L::kHalfBytes, tm_v, bars + kVFull + st, hf * 64,
+                      uc.h, t.row0, uc.b);
         ++kc_v;
       }
+      have = next_tile(p, t, t);
     }
   }
   // Drain: every issued load lands before the CTA may exit (normal path: already done).
-  if (t_ne > 0) drain_wait(q_full, (t_ne - 1) & 1);
+  if (n_q > 0) drain_wait(bars + kQFull, (n_q - 1) & 1);
   for (int st = 0; st < kStages; ++st) {
     const uint32_t uk = kc_k / kStages + (st < static_cast<int>(kc_k % kStages) ? 1u : 0u);
     const uint32_t uv = kc_v / kStages + (st < static_cast<int>(kc_v % kStages) ? 1u : 0u);
-    if (uk > 0) drain_wait(k_full + st, (uk - 1) & 1);
-    if (uv > 0) drain_wait(v_full + st, (uv - 1) & 1);
+    if (uk > 0) drain_wait(bars + kKFull + st, (uk - 1) & 1);
+    if (uv > 0) drain_wait(bars + kVFull + st, (uv - 1) & 1);
   }
 }
+
+// ------------------------------------------------------------------------------- MMA issuer
 
 template <int D>
 __device__ __forceinline__ void attn_mma(const AttnParams& p, uint8_t* smem, uint64_t* bars, uint32_t tmem,
                                          volatile int* abort_flag) {
   using L = AttnSmem<D>;
-  uint64_t* q_full = bars + 0;
-  uint64_t* q_empty = bars + 1;
-  uint64_t* k_full = bars + 2;
-  uint64_t* k_empty = bars + 4;
-  uint64_t* v_full = bars + 6;
-  uint64_t* v_empty = bars + 8;
-  uint64_t* s_full = bars + 10;
-  uint64_t* p_ready = bars + 12;
-  uint64_t* o_done = bars + 14;
-  uint64_t* o_free = bars + 15;
-  uint64_t* drain = bars + 16;
-  constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN, 0);
+  if (p.tiles_per_unit == 0) return;
+  constexpr uint32_t kIdescQK128 = idesc_bf16_f32(kBM, 128, 0);
+  constexpr uint32_t kIdescQK64 = idesc_bf16_f32(kBM, 64, 0);
   constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, D, 1);
   const uint32_t sQ = smem_u32(smem + L::kQ);
   const uint32_t sK = smem_u32(smem + L::kK);
   const uint32_t sV = smem_u32(smem + L::kV);
-  const uint32_t tmem_o = tmem + 256;
 
   uint32_t kc_k = 0, kc_v = 0;  // K/V ring positions consumed
-  uint32_t g = 0;               // global tile counter (S buffer = g & 1)
-  int t_ne = 0;
+  uint32_t g = 0;               // tiles processed (S_w / P_w phase)
+  uint32_t nch = 0;             // non-empty blocks finished (O_w phase)
+  uint32_t n_q = 0;             // units started (Q phase)
 
-  // S[g&1] = Q K_tile^T over D/16 k-steps of 16 (128B-swizzled K-major operands:
-  // step k sits in 64-column half k/4 at byte offset 32*(k%4)).
-  auto issue_qk = [&](uint32_t gg) -> bool {
-    const int st = kc_k % kStages;
-    if (!mbar_wait(k_full + st, (kc_k / kStages) & 1, abort_flag, p.status)) return false;
-    tc_fence_after();
-    const uint32_t d_tmem = tmem + (gg & 1) * kBN;
-    const uint32_t kbase = sK + st * L::kTileBytes;
+  // S_w = Q_w K^T: D/16 k-steps of 16; step k sits in 64-column half k/4 at byte 32*(k%4).
+  auto issue_qk = [&](int w, const Tile& t, int kst) {
+    const uint32_t d_tmem = tmem + w * kBN;
+    const uint32_t qbase = sQ + w * L::kTileBytes;
+    const uint32_t kbase = sK + kst * L::kTileBytes;
+    const uint32_t idesc = t.valid > 64 ? kIdescQK128 : kIdescQK64;
 #pragma unroll
     for (int k = 0; k < D / 16; ++k) {
       const uint32_t off = (k >> 2) * L::kHalfBytes + (k & 3) * 32;
-      tc_mma_ss(d_tmem, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(kbase + off, 16, 1024), kIdescQK, k > 0);
+      tc_mma_ss(d_tmem, sdesc_sw128(qbase + off, 16, 1024), sdesc_sw128(kbase + off, 16, 1024), idesc, k > 0);
     }
-    tc_commit(k_empty + st);
-    tc_commit(s_full + (gg & 1));
-    ++kc_k;
-    return true;
+    tc_commit(bars + kSFull + w);
   };
-  // O (+)= P V: P (bf16 pairs) in TMEM columns [S buffer, +64); V tile MN-major: 16 keys
-  // per k-step = 2048 bytes; the two 64-wide D halves are 16 KB apart (leading offset).
-  auto issue_pv = [&](uint32_t gg, bool accumulate) -> bool {
-    const int st = kc_v % kStages;
-    if (!mbar_wait(v_full + st, (kc_v / kStages) & 1, abort_flag, p.status)) return false;
+  // O_w (+)= P_w V: P_w (bf16 pairs) in the S_w columns; V MN-major, 16 keys per k-step
+  // = 2048 bytes; the two 64-wide D halves are 16 KB apart (leading byte offset).
+  auto issue_pv = [&](int w, const Tile& t, int vst) {
+    const uint32_t a_tmem = tmem + w * kBN;
+    const uint32_t o_tmem = tmem + 256 + w * 128;
+    const uint32_t vbase = sV + vst * L::kTileBytes;
+    const int ksteps = t.valid > 64 ? kBN / 16 : 64 / 16;
+    for (int k = 0; k < ksteps; ++k)
+      tc_mma_ts(o_tmem, a_tmem + k * 8, sdesc_sw128(vbase + k * 2048, L::kHalfBytes, 1024), kIdescPV,
+                (!t.first || k > 0) ? 1u : 0u);
+  };
+  auto wait_k = [&]() -> bool {
+    if (!mbar_wait(bars + kKFull + (kc_k % kStages), (kc_k / kStages) & 1, abort_flag, p.status)) return false;
     tc_fence_after();
-    const uint32_t a_tmem = tmem + (gg & 1) * kBN;
-    const uint32_t vbase = sV + st * L::kTileBytes;
-#pragma unroll
-    for (int k = 0; k < kBN / 16; ++k) {
-      tc_mma_ts(tmem_o, a_tmem + k * 8, sdesc_sw128(vbase + k * 2048, L::kHalfBytes, 1024), kIdescPV,
-                (accumulate || k > 0) ? 1u : 0u);
-    }
-    tc_commit(v_empty + st);
-    tc_commit(o_done);
-    ++kc_v;
     return true;
   };
 
-  for (int item = blockIdx.x; item < p.total_items; item += gridDim.x) {
-    const ItemCoord ic = decode_item(item, p);
-    const int kvlen = p.bounds[ic.c + 1] - p.bounds[ic.c];
-    const int n_kv = (kvlen + kBN - 1) / kBN;
-    if (n_kv == 0) continue;
-    if (!mbar_wait(q_full, t_ne & 1, abort_flag, p.status)) goto done;
+  for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+    if (!mbar_wait(bars + kQFull, n_q & 1, abort_flag, p.status)) goto done;
     tc_fence_after();
-    if (!issue_qk(g)) goto done;
-    if (n_kv == 1) tc_commit(q_empty);
-    for (int j = 0; j < n_kv; ++j, ++g) {
-      if (j + 1 < n_kv) {
-        if (!issue_qk(g + 1)) goto done;
-        if (j + 2 == n_kv) tc_commit(q_empty);
+    ++n_q;
+    Tile cur, nxt;
+    first_tile_from(p, 0, cur);
+    // Prologue: S for the unit's first tile, both Q tiles.
+    if (!wait_k()) goto done;
+    issue_qk(0, cur, kc_k % kStages);
+    issue_qk(1, cur, kc_k % kStages);
+    tc_commit(bars + kKEmpty + (kc_k % kStages));
+    ++kc_k;
+    bool more = next_tile(p, cur, nxt);
+    if (!more) tc_commit(bars + kQEmpty);
+    while (true) {
+      const int vst = kc_v % kStages;
+      if (!mbar_wait(bars + kVFull + vst, (kc_v / kStages) & 1, abort_flag, p.status)) goto done;
+#pragma unroll
+      for (int w = 0; w < kQTiles; ++w) {
+        if (!mbar_wait(bars + kPReady + w, g & 1, abort_flag, p.status)) goto done;
+        if (cur.first && nch > 0) {
+          if (!mbar_wait(bars + kOFree + w, (nch - 1) & 1, abort_flag, p.status)) goto done;
+        }
+        tc_fence_after();
+        issue_pv(w, cur, vst);
+        if (cur.last) tc_commit(bars + kODone + w);
+        if (more) {
+          if (w == 0 && !wait_k()) goto done;
+          issue_qk(w, nxt, kc_k % kStages);
+        }
       }
-      if (!mbar_wait(p_ready + (g & 1), (g >> 1) & 1, abort_flag, p.status)) goto done;
-      if (j == 0 && t_ne > 0) {
-        if (!mbar_wait(o_free, (t_ne - 1) & 1, abort_flag, p.status)) goto done;
+      tc_commit(bars + kVEmpty + vst);
+      ++kc_v;
+      if (more) {
+        tc_commit(bars + kKEmpty + (kc_k % kStages));
+        ++kc_k;
       }
-      tc_fence_after();
-      if (!issue_pv(g, j > 0)) goto done;
+      ++g;
+      if (cur.last) ++nch;
+      if (!more) break;
+      cur = nxt;
+      more = next_tile(p, cur, nxt);
+      if (!more) tc_commit(bars + kQEmpty);  // the unit's last QK has been issued
     }
-    ++t_ne;
   }
 done:
   // Drain: wait until every MMA this thread issued has completed.
-  tc_commit(drain);
-  drain_wait(drain, 0);
+  tc_commit(bars + kDrain);
+  drain_wait(bars + kDrain, 0);
+}
+
+// ------------------------------------------------------------------------------- softmax
+
+// Softmax of one tile of NC (128 or 64) columns for this thread's row, in one pass over
+// TMEM: the whole S row is loaded into registers (one round trip), keys at or past
+// `valid` are masked when MASK (only a block's last tile), then the row max, the lazy
+// max update, and P = 2^(S*scale*log2e - m) with packed fp32x2 FMAs, MUFU ex2 and packed
+// sums.  On return P is stored as bf16 pairs in columns [0, NC/2) of the S buffer (the
+// whole row is already in registers, so the overwrite is safe) and l/m are updated.
+template <int D, int NC, bool MASK>
+__device__ __forceinline__ void softmax_tile(uint32_t ts, uint32_t to, int valid, bool first, float sl2, float& m,
+                                             float& l) {
+  uint32_t r[NC];
+  if (NC == 128)
+    tmem_ld128(ts, *reinterpret_cast<uint32_t(*)[128]>(r));
+  else
+    tmem_ld64(ts, *reinterpret_cast<uint32_t(*)[64]>(r));
+  if (MASK) {
+#pragma unroll
+    for (int i = 0; i < NC; ++i)
+      if (i >= valid) r[i] = __float_as_uint(-INFINITY);
+  }
+  float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < NC; i += 8) {
+    a0 = fmax3(a0, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
+    a1 = fmax3(a1, __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+    a2 = fmax3(a2, __uint_as_float(r[i + 4]), __uint_as_float(r[i + 5]));
+    a3 = fmax3(a3, __uint_as_float(r[i + 6]), __uint_as_float(r[i + 7]));
+  }
+  const float m_tile = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3)) * sl2;
+  float alpha = 1.f;
+  bool rescale = false;
+  if (first) {
+    m = m_tile;
+  } else {
+    const bool need = m_tile > m + kRescaleThreshold;
+    rescale = __any_sync(0xffffffffu, need);
+    if (need) {
+      alpha = ex2_approx(m - m_tile);
+      l *= alpha;
+      m = m_tile;
+    }
+  }
+  const uint64_t scale2 = f2_pack(sl2, sl2);
+  const uint64_t negm2 = f2_pack(-m, -m);
+  uint64_t sum_a = 0, sum_b = 0;  // packed fp32 pairs (+0.0f, +0.0f)
+#pragma unroll
+  for (int c = 0; c < NC / 32; ++c) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int k = c * 32 + 2 * i;
+      const uint64_t x = fma_f32x2(f2_pack(__uint_as_float(r[k]), __uint_as_float(r[k + 1])), scale2, negm2);
+      const float p0 = ex2_approx(f2_lo(x));
+      const float p1 = ex2_approx(f2_hi(x));
+      const uint64_t pp = f2_pack(p0, p1);
+      if (i & 1)
+        sum_b = add_f32x2(sum_b, pp);
+      else
+        sum_a = add_f32x2(sum_a, pp);
+      pk[i] = pack_bf16x2(p0, p1);
+    }
+    tmem_st16(ts + c * 16, pk);
+  }
+  const uint64_t sum = add_f32x2(sum_a, sum_b);
+  l += f2_lo(sum) + f2_hi(sum);
+  if (rescale) {
+    // Rows whose max grew by more than 8 rescale O by alpha (1 for the other rows of the
+    // warp).  O holds every earlier P.V product (see the MMA issue order), and the P.V of
+    // this tile is issued only after P_ready, i.e. after these stores complete.
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t o[32];
+      tmem_ld32(to + c * 32, o);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+      tmem_st32(to + c * 32, o);
+    }
+  }
+  tmem_wait_st();
+}
+
+template <int D>
+__device__ __forceinline__ void store_row(const AttnParams& p, size_t o_off, const uint32_t (&r)[32], int c,
+                                          float inv_l) {
+  if (p.out_f32) {
+    float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out) + o_off + c * 32);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      o[i] = make_float4(__uint_as_float(r[4 * i]) * inv_l, __uint_as_float(r[4 * i + 1]) * inv_l,
+                         __uint_as_float(r[4 * i + 2]) * inv_l, __uint_as_float(r[4 * i + 3]) * inv_l);
+  } else {
+    uint4* o = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + o_off + c * 32);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      o[i] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * i + 0]) * inv_l, __uint_as_float(r[8 * i + 1]) * inv_l),
+                        pack_bf16x2(__uint_as_float(r[8 * i + 2]) * inv_l, __uint_as_float(r[8 * i + 3]) * inv_l),
+                        pack_bf16x2(__uint_as_float(r[8 * i + 4]) * inv_l, __uint_as_float(r[8 * i + 5]) * inv_l),
+                        pack_bf16x2(__uint_as_float(r[8 * i + 6]) * inv_l, __uint_as_float(r[8 * i + 7]) * inv_l));
+  }
 }
 
 template <int D>
 __device__ __forceinline__ void attn_softmax(const AttnParams& p, uint64_t* bars, uint32_t tmem,
                                              volatile int* abort_flag) {
-  uint64_t* s_full = bars + 10;
-  uint64_t* p_ready = bars + 12;
-  uint64_t* o_done = bars + 14;
-  uint64_t* o_free = bars + 15;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int quarter = warp & 3;
+  const int w = warp >> 2;        // warpgroup = Q tile of the pair
+  const int quarter = warp & 3;   // TMEM lane quarter
   const int row = quarter * 32 + lane;
-  const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-  const uint32_t taddr_o = taddr + 256;
+  const uint32_t lanes = static_cast<uint32_t>(quarter * 32) << 16;
+  const uint32_t ts = tmem + lanes + w * kBN;          // S_w
+  const uint32_t to = tmem + lanes + 256 + w * 128;    // O_w
   const float sl2 = p.scale_log2;
-  uint32_t g = 0;
+  uint32_t g = 0, nch = 0;
 
-  for (int item = blockIdx.x; item < p.total_items; item += gridDim.x) {
-    const ItemCoord ic = decode_item(item, p);
-    const int kvlen = p.bounds[ic.c + 1] - p.bounds[ic.c];
-    const int n_kv = (kvlen + kBN - 1) / kBN;
-    const int s_row = ic.qt * kBM + row;
+  for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+    const UnitCoord uc = decode_unit(u, p);
+    const int s_row = (uc.qp * kQTiles + w) * kBM + row;
     const bool row_ok = s_row < p.Sq;
-    const size_t o_off = static_cast<size_t>(ic.c) * p.out_chunk_stride +
-                         ((static_cast<size_t>(ic.b) * p.Sq + s_row) * p.H + ic.h) * D;
-    const size_t l_off = static_cast<size_t>(ic.c) * p.lse_chunk_stride +
-                         (static_cast<size_t>(ic.b) * p.H + ic.h) * p.Sq + s_row;
-    if (n_kv == 0) {  // no keys: O = 0, lse = -inf
-      if (row_ok) {
-        if (p.out_f32) {
-          float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out) + o_off);
-          for (int i = 0; i < D / 4; ++i) o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-        } else {
-          uint4* o = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + o_off);
-          for (int i = 0; i < D / 8; ++i) o[i] = make_uint4(0u, 0u, 0u, 0u);
-        }
-        if (p.lse) p.lse[l_off] = -INFINITY;
-      }
-      continue;
-    }
-
-    float m = -INFINITY;  // running max of S*scale*log2e (possibly stale by < 8)
-    float l = 0.f;        // running sum of 2^(S*scale*log2e - m)
-    for (int j = 0; j < n_kv; ++j, ++g) {
-      const uint32_t sb = g & 1;
-      if (!warp_wait(s_full + sb, (g >> 1) & 1, abort_flag, p.status)) return;
-      tc_fence_after();
-      float s[kBN];
-#pragma unroll
-      for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(taddr + sb * kBN + c * 32, r);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
-      }
-      const int valid = kvlen - j * kBN;
-      if (valid < kBN) {
-#pragma unroll
-        for (int i = 0; i < kBN; ++i)
-          if (i >= valid) s[i] = -INFINITY;
-      }
-      float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
-#pragma unroll
-      for (int i = 4; i < kBN; i += 4) {
-        mx0 = fmaxf(mx0, s[i]);
-        mx1 = fmaxf(mx1, s[i + 1]);
-        mx2 = fmaxf(mx2, s[i + 2]);
-        mx3 = fmaxf(mx3, s[i + 3]);
-      }
-      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
-      bool prev_consumed = (j == 0);
-      if (j == 0) {
-        m = m_tile;
-      } else {
-        const bool need = m_tile > m + kRescaleThreshold;
-        if (__any_sync(0xffffffffu, need)) {
-          // O must hold PV of the previous tile before it is rescaled.
-          if (!warp_wait(o_done, (g - 1) & 1, abort_flag, p.status)) return;
-          prev_consumed = true;
-          tc_fence_after();
-          const float m_new = need ? m_tile : m;
-          const float alpha = ex2_approx(m - m_new);
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t r[32];
-            tmem_ld32(taddr_o + c * 32, r);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            tmem_st32(taddr_o + c * 32, r);
+    for (int c = 0; c < p.n_chunks; ++c) {
+      const int n_kv = block_tiles(p, c);
+      if (n_kv == 0) {  // no keys: O = 0, lse = -inf
+        const size_t o_off = static_cast<size_t>(c) * p.out_chunk_stride +
+                             ((static_cast<size_t>(uc.b) * p.Sq + s_row) * p.H + uc.h) * D;
+        const size_t l_off = static_cast<size_t>(c) * p.lse_chunk_stride +
+                             (static_cast<size_t>(uc.b) * p.H + uc.h) * p.Sq + s_row;
+        if (row_ok) {
+          if (p.out_f32) {
+            float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out) + o_off);
+            for (int i = 0; i < D / 4; ++i) o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+          } else {
+            uint4* o = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + o_off);
+            for (int i = 0; i < D / 8; ++i) o[i] = make_uint4(0u, 0u, 0u, 0u);
           }
-          tmem_wait_st();
-          l *= alpha;
-          m = m_new;
+          if (p.lse) p.lse[l_off] = -INFINITY;
         }
+        continue;
       }
-      const float neg_m = -m;
-      float ls0 = 0.f, ls1 = 0.f;
-      uint32_t pk[kBN / 2];
+      float m = -INFINITY;  // running max of S*scale*log2e (possibly stale by < 8)
+      float l = 0.f;        // running sum of 2^(S*scale*log2e - m)
+      for (int j = 0; j < n_kv; ++j, ++g) {
+        const Tile t = make_tile(p, c, j);
+        if (!warp_wait(bars + kSFull + w, g & 1, abort_flag, p.status)) return;
+        tc_fence_after();
+        if (t.valid == 128)
+          softmax_tile<D, 128, false>(ts, to, t.valid, t.first, sl2, m, l);
+        else if (t.valid > 64)
+          softmax_tile<D, 128, true>(ts, to, t.valid, t.first, sl2, m, l);
+        else if (t.valid == 64)
+          softmax_tile<D, 64, false>(ts, to, t.valid, t.first, sl2, m, l);
+        else
+          softmax_tile<D, 64, true>(ts, to, t.valid, t.first, sl2, m, l);
+        tc_fence_before();
+        mbar_arrive(bars + kPReady + w);
+      }
+      // Block epilogue: wait for its last P.V, write O / l and the LSE, release O_w.
+      if (!warp_wait(bars + kODone + w, nch & 1, abort_flag, p.status)) return;
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+      const size_t o_off = static_cast<size_t>(c) * p.out_chunk_stride +
+                           ((static_cast<size_t>(uc.b) * p.Sq + s_row) * p.H + uc.h) * D;
+      const size_t l_off = static_cast<size_t>(c) * p.lse_chunk_stride +
+                           (static_cast<size_t>(uc.b) * p.H + uc.h) * p.Sq + s_row;
 #pragma unroll
-      for (int i = 0; i < kBN / 2; ++i) {
-        const float p0 = ex2_approx(fmaf(s[2 * i], sl2, neg_m));
-        const float p1 = ex2_approx(fmaf(s[2 * i + 1], sl2, neg_m));
-        ls0 += p0;
-        ls1 += p1;
-        pk[i] = pack_bf16x2(p0, p1);
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(to + cc * 32, r);
+        if (row_ok) store_row<D>(p, o_off, r, cc, inv_l);
       }
-      l += ls0 + ls1;
-#pragma unroll
-      for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t r[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) r[i] = pk[c * 16 + i];
-        tmem_st16(taddr + sb * kBN + c * 16, r);
-      }
-      tmem_wait_st();
-      // Consume PV(g-1)'s completion in order (it is long done by now).
-      if (!prev_consumed) {
-        if (!warp_wait(o_done, (g - 1) & 1, abort_flag, p.status)) return;
-      }
+      if (row_ok && p.lse) p.lse[l_off] = (m + log2f(l)) * 0.69314718055994530942f;
       tc_fence_before();
-      mbar_arrive(p_ready + sb);
+      mbar_arrive(bars + kOFree + w);
+      ++nch;
     }
-
-    // Epilogue: wait for the last PV, write O / l and the LSE, release O.
-    if (!warp_wait(o_done, (g - 1) & 1, abort_flag, p.status)) return;
-    tc_fence_after();
-    const float inv_l = 1.f / l;
-#pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-      uint32_t r[32];
-      tmem_ld32(taddr_o + c * 32, r);
-      if (row_ok) {
-        if (p.out_f32) {
-          float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out) + o_off + c * 32);
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            o[i] = make_float4(__uint_as_float(r[4 * i]) * inv_l, __uint_as_float(r[4 * i + 1]) * inv_l,
-                               __uint_as_float(r[4 * i + 2]) * inv_l, __uint_as_float(r[4 * i + 3]) * inv_l);
-        } else {
-          uint4* o = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + o_off + c * 32);
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            o[i] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * i + 0]) * inv_l, __uint_as_float(r[8 * i + 1]) * inv_l),
-                              pack_bf16x2(__uint_as_float(r[8 * i + 2]) * inv_l, __uint_as_float(r[8 * i + 3]) * inv_l),
-                              pack_bf16x2(__uint_as_float(r[8 * i + 4]) * inv_l, __uint_as_float(r[8 * i + 5]) * inv_l),
-                              pack_bf16x2(__uint_as_float(r[8 * i + 6]) * inv_l, __uint_as_float(r[8 * i + 7]) * inv_l));
-        }
-      }
-    }
-    if (row_ok && p.lse) p.lse[l_off] = (m + log2f(l)) * 0.69314718055994530942f;
-    tc_fence_before();
-    mbar_arrive(o_free);
   }
 }
+
+// ------------------------------------------------------------------------------- kernel
 
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1)
@@ -421,31 +515,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int warp = threadIdx.x >> 5;
 
   if (threadIdx.x == 0) {
-    mbar_init(bars + 0, 1);   // q_full (TMA tx)
-    mbar_init(bars + 1, 1);   // q_empty (MMA commit)
+    mbar_init(bars + kQFull, 1);    // TMA transaction count
+    mbar_init(bars + kQEmpty, 1);   // MMA commit
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(bars + 2 + s, 1);  // k_full
-      mbar_init(bars + 4 + s, 1);  // k_empty
-      mbar_init(bars + 6 + s, 1);  // v_full
-      mbar_init(bars + 8 + s, 1);  // v_empty
+      mbar_init(bars + kKFull + s, 1);
+      mbar_init(bars + kKEmpty + s, 1);
+      mbar_init(bars + kVFull + s, 1);
+      mbar_init(bars + kVEmpty + s, 1);
     }
-    mbar_init(bars + 10, 1);   // s_full[0]
-    mbar_init(bars + 11, 1);   // s_full[1]
-    mbar_init(bars + 12, 128); // p_ready[0] (softmax threads)
-    mbar_init(bars + 13, 128); // p_ready[1]
-    mbar_init(bars + 14, 1);   // o_done (MMA commit after each PV)
-    mbar_init(bars + 15, 128); // o_free (softmax epilogue done with O)
-    mbar_init(bars + 16, 1);   // drain
+    for (int w = 0; w < kQTiles; ++w) {
+      mbar_init(bars + kSFull + w, 1);     // MMA commit after QK_w
+      mbar_init(bars + kPReady + w, 128);  // the 128 threads of softmax warpgroup w
+      mbar_init(bars + kODone + w, 1);     // MMA commit after a block's last PV_w
+      mbar_init(bars + kOFree + w, 128);   // warpgroup w has read O_w
+    }
+    mbar_init(bars + kDrain, 1);
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
   }
-  if (warp == 0 && (threadIdx.x & 31) == 0) {
+  if (warp == kProducerWarp && (threadIdx.x & 31) == 0) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
   }
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
@@ -456,20 +550,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   // Producer and MMA roles run on lane 0 of their warp; the other lanes wait at the
   // __syncwarp so that each warp is converged again for the teardown below.
-  if (warp == 0) {
-    if ((threadIdx.x & 31) == 0) attn_producer<D>(&tm_q, &tm_k, &tm_v, p, smem, bars, abort_flag);
-    __syncwarp();
-  } else if (warp == 1) {
-    if ((threadIdx.x & 31) == 0) attn_mma<D>(p, smem, bars, tmem, abort_flag);
+  // Warps 10 and 11 only give their registers back to the softmax warpgroups.
+  if (warp >= kQTiles * 4) {
+    regs_decrease<kControlRegs>();
+    if (warp == kProducerWarp) {
+      if ((threadIdx.x & 31) == 0) attn_producer<D>(&tm_q, &tm_k, &tm_v, p, smem, bars, abort_flag);
+    } else if (warp == kMmaWarp) {
+      if ((threadIdx.x & 31) == 0) attn_mma<D>(p, smem, bars, tmem, abort_flag);
+    }
     __syncwarp();
   } else {
+    regs_increase<kSoftmaxRegs>();
     attn_softmax<D>(p, bars, tmem, abort_flag);
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+  if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
 }  // namespace cpattn

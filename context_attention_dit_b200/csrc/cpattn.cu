@@ -92,9 +92,11 @@ cp_status check_attn_args(const void* q, const void* k, const void* v, const voi
   if (!aligned16(q) || !aligned16(out) || (Skv > 0 && (!aligned16(k) || !aligned16(v))) ||
       (lse && !aligned16(lse)))
     return CP_ERR_MISALIGNED;
-  // 32-bit limits: TMA coordinates, item counts.
+  // 32-bit limits: TMA coordinates, unit counts.
   const long long n_qt = (Sq + kBM - 1) / kBM;
-  if (static_cast<long long>(B) * H * n_qt * kMaxChunks >= (1LL << 31)) return CP_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H * n_qt >= (1LL << 31) || static_cast<long long>(Sq) + 2 * kBM >= (1LL << 31) ||
+      static_cast<long long>(Skv) + kBN >= (1LL << 31))
+    return CP_ERR_UNSUPPORTED;
   return CP_OK;
 }
 
@@ -111,8 +113,10 @@ cp_status launch_attn(const void* q, const void* k, const void* v, const int* bo
   p.H = H;
   p.Sq = Sq;
   p.n_chunks = n_chunks;
-  p.n_qt = (Sq + kBM - 1) / kBM;
-  p.total_items = B * H * n_chunks * p.n_qt;
+  p.n_qp = (Sq + kQTiles * kBM - 1) / (kQTiles * kBM);
+  p.n_units = B * H * p.n_qp;
+  p.tiles_per_unit = 0;
+  for (int i = 0; i < n_chunks; ++i) p.tiles_per_unit += (bounds[i + 1] - bounds[i] + kBN - 1) / kBN;
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.out = out;
   p.out_f32 = out_f32;
@@ -131,7 +135,7 @@ cp_status launch_attn(const void* q, const void* k, const void* v, const int* bo
       make_bshd_map(&tv, vp, B, Skv > 0 ? kv_rows : Sq, H, D) != CP_OK)
     return CP_ERR_CUDA;
 
-  const int grid = p.total_items < dev->num_sms ? p.total_items : dev->num_sms;
+  const int grid = p.n_units < dev->num_sms ? p.n_units : dev->num_sms;
   if (D == 128) {
     using L = AttnSmem<128>;
     if (!dev->attn_attr_set[1]) {
