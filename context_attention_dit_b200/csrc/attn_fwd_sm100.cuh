@@ -14,10 +14,12 @@
 //               Per K/V tile: load the S row from TMEM, mask keys past the block end,
 //               update the running max m and sum l (base 2), write P = 2^(S*scale*log2e
 //               - m) as bf16 pairs into the first columns of the same S buffer.  After
-//               a block's last tile: write O/l (fp32 partial or final bf16/fp32) and lse.
+//               a block's last tile: hand the row's (m, l) to the epilogue warpgroup.
 //   warp 8      TMA producer: both Q tiles once per unit; K and V tiles (128 keys x D)
 //               through two 2-stage rings.  Warps 8-11 form the control warpgroup, which
-//               hands registers to the softmax warpgroups (setmaxnreg 88 / 208).
+//               hands registers to the softmax warpgroups (setmaxnreg 88 / 184 / 56).
+//   warps 12-15 epilogue warpgroup: after a block's last P.V, read O_w from TMEM, release
+//               it for the next block, write O/l (fp32 partial or final bf16/fp32) and lse.
 //   warp 9      TMEM owner (512 columns) and MMA issuer (one thread), in the order
 //               QK0(t) QK1(t) | PV0(t) QK0(t+1) PV1(t) QK1(t+1) | ...
 //               S_w = Q_w K^T: SS form, both operands K-major and 128B-swizzled;
@@ -45,13 +47,16 @@ constexpr int kBM = 128;           // query rows per Q tile (TMEM lanes)
 constexpr int kQTiles = 2;         // Q tiles per work unit, one softmax warpgroup each
 constexpr int kBN = 128;           // keys per K/V tile
 constexpr int kStages = 2;         // stages of each of the K and V rings
-constexpr int kAttnThreads = 384;  // 12 warps: two softmax warpgroups + a control warpgroup
+constexpr int kAttnThreads = 512;  // 16 warps: 2 softmax, 1 control, 1 epilogue warpgroup
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
-// Registers per thread after the split (launch: 168 = 65536 / 384 rounded down to 8).
-// 256 * 208 + 128 * 88 = 384 * 168.
-constexpr int kSoftmaxRegs = 208;
+constexpr int kEpilogueWarp0 = 12;
+// Registers per thread after the split (launch: 128 = 65536 / 512).
+// 256 * kSoftmaxRegs + 128 * kControlRegs + 128 * kEpilogueRegs = 512 * 128.
+constexpr int kSoftmaxRegs = 184;
 constexpr int kControlRegs = 88;
+constexpr int kEpilogueRegs = 56;
+static_assert(2 * kSoftmaxRegs + kControlRegs + kEpilogueRegs == 4 * 128, "register split must use the launch budget");
 constexpr int kTmemCols = 512;
 constexpr int kMaxChunks = 64;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -79,8 +84,9 @@ struct AttnSmem {
   static constexpr int kQ = 0;                     // kQTiles Q tiles
   static constexpr int kK = kQ + kQTiles * kTileBytes;
   static constexpr int kV = kK + kStages * kTileBytes;
-  static constexpr int kBar = kV + kStages * kTileBytes;
-  static constexpr int kNumBars = 19;
+  static constexpr int kStat = kV + kStages * kTileBytes;  // float2 [kQTiles][2][kBM]: (m, l) per row
+  static constexpr int kBar = kStat + kQTiles * 2 * kBM * 8;
+  static constexpr int kNumBars = 21;
   static constexpr int kUsed = kBar + kNumBars * 8 + 16;
   // More than half an SM's shared memory: exactly one CTA (owning all 512 TMEM
   // columns) is resident per SM.
@@ -90,7 +96,7 @@ struct AttnSmem {
 // Barrier indices.
 enum : int {
   kQFull = 0, kQEmpty = 1, kKFull = 2, kKEmpty = 4, kVFull = 6, kVEmpty = 8,
-  kSFull = 10, kPReady = 12, kODone = 14, kOFree = 16, kDrain = 18
+  kSFull = 10, kPReady = 12, kODone = 14, kOFree = 16, kStatReady = 18, kDrain = 20
 };
 
 struct UnitCoord {
@@ -425,8 +431,27 @@ __device__ __forceinline__ void store_row(const AttnParams& p, size_t o_off, con
 }
 
 template <int D>
-__device__ __forceinline__ void attn_softmax(const AttnParams& p, uint64_t* bars, uint32_t tmem,
+__device__ __forceinline__ void write_empty_row(const AttnParams& p, int c, const UnitCoord& uc, int s_row) {
+  const size_t o_off = static_cast<size_t>(c) * p.out_chunk_stride +
+                       ((static_cast<size_t>(uc.b) * p.Sq + s_row) * p.H + uc.h) * D;
+  if (p.out_f32) {
+    float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out) + o_off);
+    for (int i = 0; i < D / 4; ++i) o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  } else {
+    uint4* o = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + o_off);
+    for (int i = 0; i < D / 8; ++i) o[i] = make_uint4(0u, 0u, 0u, 0u);
+  }
+  if (p.lse)
+    p.lse[static_cast<size_t>(c) * p.lse_chunk_stride + (static_cast<size_t>(uc.b) * p.H + uc.h) * p.Sq + s_row] =
+        -INFINITY;
+}
+
+// Softmax warpgroup w: every tile of every block of every unit; at a block's end it hands
+// the row's (m, l) to the epilogue warpgroup and carries on with the next block.
+template <int D>
+__device__ __forceinline__ void attn_softmax(const AttnParams& p, uint8_t* smem, uint64_t* bars, uint32_t tmem,
                                              volatile int* abort_flag) {
+  using L = AttnSmem<D>;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int w = warp >> 2;        // warpgroup = Q tile of the pair
@@ -435,30 +460,17 @@ __device__ __forceinline__ void attn_softmax(const AttnParams& p, uint64_t* bars
   const uint32_t lanes = static_cast<uint32_t>(quarter * 32) << 16;
   const uint32_t ts = tmem + lanes + w * kBN;          // S_w
   const uint32_t to = tmem + lanes + 256 + w * 128;    // O_w
+  float2* stat = reinterpret_cast<float2*>(smem + L::kStat) + w * 2 * kBM;
   const float sl2 = p.scale_log2;
   uint32_t g = 0, nch = 0;
 
   for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
     const UnitCoord uc = decode_unit(u, p);
     const int s_row = (uc.qp * kQTiles + w) * kBM + row;
-    const bool row_ok = s_row < p.Sq;
     for (int c = 0; c < p.n_chunks; ++c) {
       const int n_kv = block_tiles(p, c);
       if (n_kv == 0) {  // no keys: O = 0, lse = -inf
-        const size_t o_off = static_cast<size_t>(c) * p.out_chunk_stride +
-                             ((static_cast<size_t>(uc.b) * p.Sq + s_row) * p.H + uc.h) * D;
-        const size_t l_off = static_cast<size_t>(c) * p.lse_chunk_stride +
-                             (static_cast<size_t>(uc.b) * p.H + uc.h) * p.Sq + s_row;
-        if (row_ok) {
-          if (p.out_f32) {
-            float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out) + o_off);
-            for (int i = 0; i < D / 4; ++i) o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-          } else {
-            uint4* o = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + o_off);
-            for (int i = 0; i < D / 8; ++i) o[i] = make_uint4(0u, 0u, 0u, 0u);
-          }
-          if (p.lse) p.lse[l_off] = -INFINITY;
-        }
+        if (s_row < p.Sq) write_empty_row<D>(p, c, uc, s_row);
         continue;
       }
       float m = -INFINITY;  // running max of S*scale*log2e (possibly stale by < 8)
@@ -478,23 +490,61 @@ __device__ __forceinline__ void attn_softmax(const AttnParams& p, uint64_t* bars
         tc_fence_before();
         mbar_arrive(bars + kPReady + w);
       }
-      // Block epilogue: wait for its last P.V, write O / l and the LSE, release O_w.
-      if (!warp_wait(bars + kODone + w, nch & 1, abort_flag, p.status)) return;
-      tc_fence_after();
-      const float inv_l = 1.f / l;
-      const size_t o_off = static_cast<size_t>(c) * p.out_chunk_stride +
-                           ((static_cast<size_t>(uc.b) * p.Sq + s_row) * p.H + uc.h) * D;
-      const size_t l_off = static_cast<size_t>(c) * p.lse_chunk_stride +
-                           (static_cast<size_t>(uc.b) * p.H + uc.h) * p.Sq + s_row;
+      // Hand (m, l) of this block to the epilogue warpgroup.  First wait until the epilogue
+      // has finished the previous block (it releases O_w only after reading that block's
+      // stats): without this wait, blocks of a single tile let this warpgroup run two
+      // stat_ready phases ahead of the epilogue, which a parity wait cannot tell apart.
+      if (nch > 0 && !warp_wait(bars + kOFree + w, (nch - 1) & 1, abort_flag, p.status)) return;
+      stat[(nch & 1) * kBM + row] = make_float2(m, l);
+      mbar_arrive(bars + kStatReady + w);
+      ++nch;
+    }
+  }
+}
+
+// Epilogue warpgroup: for every non-empty block and both Q tiles, wait for the block's
+// last P.V and its (m, l), read O_w from TMEM 32 columns at a time, write O/l and the LSE,
+// then release O_w for the next block's first P.V.
+template <int D>
+__device__ __forceinline__ void attn_epilogue(const AttnParams& p, uint8_t* smem, uint64_t* bars, uint32_t tmem,
+                                              volatile int* abort_flag) {
+  using L = AttnSmem<D>;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int quarter = warp & 3;
+  const int row = quarter * 32 + lane;
+  const uint32_t lanes = static_cast<uint32_t>(quarter * 32) << 16;
+  const float2* stat = reinterpret_cast<const float2*>(smem + L::kStat);
+  uint32_t nch = 0;
+  if (p.tiles_per_unit == 0) return;
+  for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+    const UnitCoord uc = decode_unit(u, p);
+    for (int c = 0; c < p.n_chunks; ++c) {
+      if (block_tiles(p, c) == 0) continue;
+#pragma unroll 1
+      for (int w = 0; w < kQTiles; ++w) {
+        if (!warp_wait(bars + kStatReady + w, nch & 1, abort_flag, p.status)) return;
+        if (!warp_wait(bars + kODone + w, nch & 1, abort_flag, p.status)) return;
+        tc_fence_after();
+        const float2 ml = stat[(w * 2 + (nch & 1)) * kBM + row];
+        const float inv_l = 1.f / ml.y;
+        const int s_row = (uc.qp * kQTiles + w) * kBM + row;
+        const bool row_ok = s_row < p.Sq;
+        const size_t o_off = static_cast<size_t>(c) * p.out_chunk_stride +
+                             ((static_cast<size_t>(uc.b) * p.Sq + s_row) * p.H + uc.h) * D;
+        const uint32_t to = tmem + lanes + 256 + w * 128;
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t r[32];
-        tmem_ld32(to + cc * 32, r);
-        if (row_ok) store_row<D>(p, o_off, r, cc, inv_l);
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t r[32];
+          tmem_ld32(to + cc * 32, r);
+          if (row_ok) store_row<D>(p, o_off, r, cc, inv_l);
+        }
+        tc_fence_before();
+        mbar_arrive(bars + kOFree + w);
+        if (row_ok && p.lse)
+          p.lse[static_cast<size_t>(c) * p.lse_chunk_stride + (static_cast<size_t>(uc.b) * p.H + uc.h) * p.Sq +
+                s_row] = (ml.x + log2f(ml.y)) * 0.69314718055994530942f;
       }
-      if (row_ok && p.lse) p.lse[l_off] = (m + log2f(l)) * 0.69314718055994530942f;
-      tc_fence_before();
-      mbar_arrive(bars + kOFree + w);
       ++nch;
     }
   }
@@ -527,7 +577,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(bars + kSFull + w, 1);     // MMA commit after QK_w
       mbar_init(bars + kPReady + w, 128);  // the 128 threads of softmax warpgroup w
       mbar_init(bars + kODone + w, 1);     // MMA commit after a block's last PV_w
-      mbar_init(bars + kOFree + w, 128);   // warpgroup w has read O_w
+      mbar_init(bars + kOFree + w, 128);   // the epilogue warpgroup has read O_w
+      mbar_init(bars + kStatReady + w, 128);  // warpgroup w has written a block's (m, l)
     }
     mbar_init(bars + kDrain, 1);
     *abort_flag = 0;
@@ -551,7 +602,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   // Producer and MMA roles run on lane 0 of their warp; the other lanes wait at the
   // __syncwarp so that each warp is converged again for the teardown below.
   // Warps 10 and 11 only give their registers back to the softmax warpgroups.
-  if (warp >= kQTiles * 4) {
+  if (warp >= kEpilogueWarp0) {
+    regs_decrease<kEpilogueRegs>();
+    attn_epilogue<D>(p, smem, bars, tmem, abort_flag);
+  } else if (warp >= kQTiles * 4) {
     regs_decrease<kControlRegs>();
     if (warp == kProducerWarp) {
       if ((threadIdx.x & 31) == 0) attn_producer<D>(&tm_q, &tm_k, &tm_v, p, smem, bars, abort_flag);
@@ -561,7 +615,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     __syncwarp();
   } else {
     regs_increase<kSoftmaxRegs>();
-    attn_softmax<D>(p, bars, tmem, abort_flag);
+    attn_softmax<D>(p, smem, bars, tmem, abort_flag);
   }
 
   tc_fence_before();
