@@ -158,14 +158,12 @@ def run_ours(args):
     flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
     scale = w.scale
     flop = w.flop
-    launches_per_step = 3 + 2 + 1
+    launches_per_step = 1 + 2 + 1  # permute (Q,K,V), attention, merge, inverse permute
 
     def step(evs=None):
         if evs:
             evs[0].record()
-        binding.ulysses_permute(xq, P, 0, dst=yq)
-        binding.ulysses_permute(xk, P, 0, dst=yk)
-        binding.ulysses_permute(xv, P, 0, dst=yv)
+        binding.ulysses_permute_n((xq, xk, xv), P, 0, dsts=(yq, yk, yv))
         if evs:
             evs[1].record()
         view = lambda t: t.view(Bp, S, Hp, D)
@@ -434,9 +432,9 @@ def run_profile_case(args):
             lses = torch.randn(8, B, H, S, device="cuda")
             binding.attn_merge(parts, lses)
         elif case == "permute":
-            x = q.view(B, P, S // P, H, D).permute(1, 0, 2, 3, 4).contiguous()
-            y = binding.ulysses_permute(x, P, 0)
-            binding.ulysses_permute(y, P, 1)
+            xs = [t.view(B, P, S // P, H, D).permute(1, 0, 2, 3, 4).contiguous() for t in (q, k, v)]
+            ys = binding.ulysses_permute_n(xs, P, 0)
+            binding.ulysses_permute(ys[0], P, 1)
     torch.cuda.synchronize()
     assert binding.last_device_status() == 0
     print(f"profile case {case} x{args.profile_reps} batch {B}: ok")

@@ -18,9 +18,10 @@ from .binding import (  # noqa: F401
     ring_workspace_views,
     status_string,
     ulysses_permute,
+    ulysses_permute_n,
 )
 
 __all__ = [
     "CpError", "attn_fwd", "attn_fwd_blocks", "attn_merge", "last_device_status", "load", "ring_bounds", "ring_sim",
-    "ring_workspace_size", "ring_workspace_views", "status_string", "ulysses_permute",
+    "ring_workspace_size", "ring_workspace_views", "status_string", "ulysses_permute", "ulysses_permute_n",
 ]

@@ -33,7 +33,7 @@ CP_MAX_CHUNKS = 64
 
 EXPORTS = (
     "cp_attn_fwd", "cp_attn_fwd_blocks", "cp_attn_merge", "cp_ring_sim_workspace_size", "cp_ring_sim", "cp_ulysses_permute",
-    "cp_ring_bounds", "cp_last_device_status", "cp_status_string", "cp_version",
+    "cp_ulysses_permute_n", "cp_ring_bounds", "cp_last_device_status", "cp_status_string", "cp_version",
 )
 
 _lib = None
@@ -63,6 +63,8 @@ def load() -> ctypes.CDLL:
     lib.cp_ring_sim.argtypes = [vp, vp, vp, ip, i, vp, vp, i, i, i, i, i, f, i, vp, sz, vp]
     lib.cp_ring_sim_static.argtypes = [vp, vp, vp, ip, i, vp, vp, i, i, i, i, i, f, i, vp]
     lib.cp_ulysses_permute.argtypes = [vp, vp, i, i, i, i, i, i, i, vp]
+    lib.cp_ulysses_permute_n.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), i, i, i, i, i, i, i, i, vp]
+    lib.cp_ulysses_permute_n.restype = ctypes.c_int
     lib.cp_ring_bounds.argtypes = [i, i, i, ip]
     lib.cp_last_device_status.argtypes = [vp]
     lib.cp_status_string.argtypes = [i]
@@ -278,6 +280,46 @@ def ulysses_permute(src, degree: int, direction: int, dst=None):
                                    ctypes.c_void_p(_stream(src)))
     _check(st, "cp_ulysses_permute")
     return dst
+
+
+def ulysses_permute_n(srcs, degree: int, direction: int, dsts=None):
+    """Ulysses exchange of several same-shaped tensors (e.g. Q, K, V) in one launch."""
+    srcs = list(srcs)
+    if not srcs:
+        raise ValueError("need at least one tensor")
+    ref = srcs[0]
+    for t in srcs:
+        if not t.is_cuda or not t.is_contiguous() or t.shape != ref.shape or t.dtype != ref.dtype \
+                or t.device != ref.device:
+            raise ValueError("tensors must be contiguous CUDA tensors of one shape, dtype and device")
+    if dsts is None:
+        dsts = [None] * len(srcs)
+    dsts = list(dsts)
+    P = int(degree)
+    if ref.dim() != 5 or ref.shape[0] != P:
+        raise ValueError(f"src must be 5-D with leading dim {P}, got {tuple(ref.shape)}")
+    if direction == 0:
+        _, B, Sp, H, D = ref.shape
+        S = Sp * P
+        if H % P:
+            raise ValueError(f"heads {H} not divisible by degree {P}")
+        shape = (P, B, S, H // P, D)
+    elif direction == 1:
+        _, B, S, Hp, D = ref.shape
+        H = Hp * P
+        if S % P:
+            raise ValueError(f"sequence {S} not divisible by degree {P}")
+        shape = (P, B, S // P, H, D)
+    else:
+        raise ValueError("direction must be 0 or 1")
+    dsts = [torch.empty(shape, dtype=ref.dtype, device=ref.device) if d is None else d for d in dsts]
+    n = len(srcs)
+    sp = (ctypes.c_void_p * n)(*[t.data_ptr() for t in srcs])
+    dp = (ctypes.c_void_p * n)(*[t.data_ptr() for t in dsts])
+    st = load().cp_ulysses_permute_n(sp, dp, n, P, B, S, H, D, direction, ref.element_size(),
+                                     ctypes.c_void_p(_stream(ref)))
+    _check(st, "cp_ulysses_permute_n")
+    return dsts
 
 
 def ring_bounds(S: int, n: int, anything: bool = False):

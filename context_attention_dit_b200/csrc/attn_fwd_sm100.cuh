@@ -70,6 +70,7 @@ struct AttnParams {
   float scale_log2;          // scale * log2(e)
   void* out;                 // block c at out + c*out_chunk_stride elements, [B][Sq][H][D]
   int out_f32;               // 1: fp32 output, 0: bf16 output
+  int out_v8;                // 1: out is 32-byte aligned (32-byte stores)
   long long out_chunk_stride;
   float* lse;                // block c at lse + c*lse_chunk_stride, [B][H][Sq]; may be null
   long long lse_chunk_stride;
@@ -410,23 +411,41 @@ __device__ __forceinline__ void softmax_tile(uint32_t ts, uint32_t to, int valid
   tmem_wait_st();
 }
 
+// Write 32 columns (block cc) of this thread's output row, scaled by 1/l: fp32 or bf16,
+// with 32-byte stores when the output base is 32-byte aligned (p.out_v8), else 16-byte.
 template <int D>
-__device__ __forceinline__ void store_row(const AttnParams& p, size_t o_off, const uint32_t (&r)[32], int c,
+__device__ __forceinline__ void store_row(const AttnParams& p, size_t o_off, const uint32_t (&r)[32], int cc,
                                           float inv_l) {
+  auto sc = [&](int i) { return __uint_as_float(r[i]) * inv_l; };
   if (p.out_f32) {
-    float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out) + o_off + c * 32);
+    float* o = static_cast<float*>(p.out) + o_off + cc * 32;
+    if (p.out_v8) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-      o[i] = make_float4(__uint_as_float(r[4 * i]) * inv_l, __uint_as_float(r[4 * i + 1]) * inv_l,
-                         __uint_as_float(r[4 * i + 2]) * inv_l, __uint_as_float(r[4 * i + 3]) * inv_l);
+      for (int i = 0; i < 4; ++i)
+        st_global_v8(o + 8 * i, __float_as_uint(sc(8 * i)), __float_as_uint(sc(8 * i + 1)),
+                     __float_as_uint(sc(8 * i + 2)), __float_as_uint(sc(8 * i + 3)), __float_as_uint(sc(8 * i + 4)),
+                     __float_as_uint(sc(8 * i + 5)), __float_as_uint(sc(8 * i + 6)), __float_as_uint(sc(8 * i + 7)));
+    } else {
+      float4* o4 = reinterpret_cast<float4*>(o);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o4[i] = make_float4(sc(4 * i), sc(4 * i + 1), sc(4 * i + 2), sc(4 * i + 3));
+    }
   } else {
-    uint4* o = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + o_off + c * 32);
+    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + o_off + cc * 32;
+    if (p.out_v8) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      o[i] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * i + 0]) * inv_l, __uint_as_float(r[8 * i + 1]) * inv_l),
-                        pack_bf16x2(__uint_as_float(r[8 * i + 2]) * inv_l, __uint_as_float(r[8 * i + 3]) * inv_l),
-                        pack_bf16x2(__uint_as_float(r[8 * i + 4]) * inv_l, __uint_as_float(r[8 * i + 5]) * inv_l),
-                        pack_bf16x2(__uint_as_float(r[8 * i + 6]) * inv_l, __uint_as_float(r[8 * i + 7]) * inv_l));
+      for (int i = 0; i < 2; ++i)
+        st_global_v8(o + 16 * i, pack_bf16x2(sc(16 * i + 0), sc(16 * i + 1)), pack_bf16x2(sc(16 * i + 2), sc(16 * i + 3)),
+                     pack_bf16x2(sc(16 * i + 4), sc(16 * i + 5)), pack_bf16x2(sc(16 * i + 6), sc(16 * i + 7)),
+                     pack_bf16x2(sc(16 * i + 8), sc(16 * i + 9)), pack_bf16x2(sc(16 * i + 10), sc(16 * i + 11)),
+                     pack_bf16x2(sc(16 * i + 12), sc(16 * i + 13)), pack_bf16x2(sc(16 * i + 14), sc(16 * i + 15)));
+    } else {
+      uint4* o4 = reinterpret_cast<uint4*>(o);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        o4[i] = make_uint4(pack_bf16x2(sc(8 * i + 0), sc(8 * i + 1)), pack_bf16x2(sc(8 * i + 2), sc(8 * i + 3)),
+                           pack_bf16x2(sc(8 * i + 4), sc(8 * i + 5)), pack_bf16x2(sc(8 * i + 6), sc(8 * i + 7)));
+    }
   }
 }
 

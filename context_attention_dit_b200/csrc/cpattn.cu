@@ -120,6 +120,7 @@ cp_status launch_attn(const void* q, const void* k, const void* v, const int* bo
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.out = out;
   p.out_f32 = out_f32;
+  p.out_v8 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0 ? 1 : 0;
   p.out_chunk_stride = out_chunk_stride;
   p.lse = lse;
   p.lse_chunk_stride = lse_chunk_stride;
@@ -327,35 +328,49 @@ cp_status cp_ring_sim_static(const void* q, const void* k, const void* v, const 
                      need, stream);
 }
 
-cp_status cp_ulysses_permute(const void* src, void* dst, int degree, int B, int S, int H, int D, int direction,
-                             int elem_bytes, void* stream) {
+cp_status cp_ulysses_permute_n(const void* const* srcs, void* const* dsts, int n_tensors, int degree, int B, int S,
+                               int H, int D, int direction, int elem_bytes, void* stream) {
   if (degree < 1 || B < 0 || S < 0 || H < 0 || D < 0) return CP_ERR_INVALID_ARG;
   if (direction != 0 && direction != 1) return CP_ERR_INVALID_ARG;
   if (elem_bytes != 2 && elem_bytes != 4) return CP_ERR_UNSUPPORTED;
+  if (n_tensors < 1 || !srcs || !dsts) return CP_ERR_INVALID_ARG;
+  if (n_tensors > kPermuteMaxTensors) return CP_ERR_UNSUPPORTED;
   if (S % degree != 0 || H % degree != 0) return CP_ERR_NOT_DIVISIBLE;
   if (B == 0 || S == 0 || H == 0 || D == 0) return CP_OK;
-  if (!src || !dst) return CP_ERR_INVALID_ARG;
-  if (!aligned16(src) || !aligned16(dst)) return CP_ERR_MISALIGNED;
   const long long row_bytes = static_cast<long long>(H) * D * elem_bytes;
   const long long piece_bytes = row_bytes / degree;
   const long long total = static_cast<long long>(B) * S * row_bytes;
-  const char* s0 = static_cast<const char*>(src);
-  const char* d0 = static_cast<const char*>(dst);
-  if (s0 < d0 + total && d0 < s0 + total) return CP_ERR_INVALID_ARG;  // overlap
-  if (static_cast<long long>(degree) * B > 65535 || row_bytes / 2 >= (1LL << 31)) return CP_ERR_UNSUPPORTED;
+  PermuteArgs a;
+  for (int t = 0; t < n_tensors; ++t) {
+    if (!srcs[t] || !dsts[t]) return CP_ERR_INVALID_ARG;
+    if (!aligned16(srcs[t]) || !aligned16(dsts[t])) return CP_ERR_MISALIGNED;
+    a.src[t] = srcs[t];
+    a.dst[t] = dsts[t];
+  }
+  // No destination may overlap any source or another destination.
+  for (int t = 0; t < n_tensors; ++t) {
+    const char* d0 = static_cast<const char*>(dsts[t]);
+    for (int u = 0; u < n_tensors; ++u) {
+      const char* s0 = static_cast<const char*>(srcs[u]);
+      if (s0 < d0 + total && d0 < s0 + total) return CP_ERR_INVALID_ARG;
+      const char* e0 = static_cast<const char*>(dsts[u]);
+      if (u != t && e0 < d0 + total && d0 < e0 + total) return CP_ERR_INVALID_ARG;
+    }
+  }
+  if (static_cast<long long>(n_tensors) * degree * B > 65535 || row_bytes / 2 >= (1LL << 31)) return CP_ERR_UNSUPPORTED;
   DeviceInfo* dev = nullptr;
   cp_status st = device_info(&dev);
   if (st != CP_OK) return st;
   const int Sp = S / degree;
-  const unsigned gy = static_cast<unsigned>(Sp < 65535 ? Sp : 65535);
+  const int groups = (Sp + kPermuteRows - 1) / kPermuteRows;
+  const unsigned gy = static_cast<unsigned>(groups < 65535 ? groups : 65535);
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   auto launch = [&](auto tag) {
     using V = decltype(tag);
     const int row_vecs = static_cast<int>(row_bytes / sizeof(V));
     const int piece_vecs = static_cast<int>(piece_bytes / sizeof(V));
-    const dim3 grid((row_vecs + kPermuteThreads - 1) / kPermuteThreads, gy, degree * B);
-    ulysses_permute_kernel<V><<<grid, kPermuteThreads, 0, cs>>>(static_cast<const V*>(src), static_cast<V*>(dst),
-                                                                degree, B, Sp, row_vecs, piece_vecs, direction);
+    const dim3 grid((row_vecs + kPermuteThreads - 1) / kPermuteThreads, gy, n_tensors * degree * B);
+    ulysses_permute_kernel<V><<<grid, kPermuteThreads, 0, cs>>>(a, degree, B, Sp, row_vecs, piece_vecs, direction);
   };
   if (piece_bytes % 16 == 0)
     launch(uint4{});
@@ -366,6 +381,18 @@ cp_status cp_ulysses_permute(const void* src, void* dst, int degree, int B, int 
   else
     launch(uint16_t{});
   return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+}
+
+cp_status cp_ulysses_permute(const void* src, void* dst, int degree, int B, int S, int H, int D, int direction,
+                             int elem_bytes, void* stream) {
+  // Pointers are checked by the batched form; nulls with empty sizes stay a no-op.
+  if (degree < 1 || B < 0 || S < 0 || H < 0 || D < 0) return CP_ERR_INVALID_ARG;
+  if (direction != 0 && direction != 1) return CP_ERR_INVALID_ARG;
+  if (elem_bytes != 2 && elem_bytes != 4) return CP_ERR_UNSUPPORTED;
+  if (S % degree != 0 || H % degree != 0) return CP_ERR_NOT_DIVISIBLE;
+  if (B == 0 || S == 0 || H == 0 || D == 0) return CP_OK;
+  if (!src || !dst) return CP_ERR_INVALID_ARG;
+  return cp_ulysses_permute_n(&src, &dst, 1, degree, B, S, H, D, direction, elem_bytes, stream);
 }
 
 cp_status cp_ring_bounds(int S, int n, int anything, int* bounds_out) {

@@ -185,6 +185,17 @@ CP_API cp_status cp_ulysses_permute(const void* src, void* dst, int degree, int 
                              int direction, int elem_bytes, void* stream);
 
 /*
+ * cp_ulysses_permute_n - cp_ulysses_permute of n_tensors same-shaped tensors in one
+ * launch (the Ulysses exchange moves Q, K and V together).
+ *
+ * srcs, dsts: HOST arrays of n_tensors device pointers (1 <= n_tensors <= 8), read during
+ * the call only.  Other arguments and rules as cp_ulysses_permute; no destination may
+ * overlap any source or another destination (CP_ERR_INVALID_ARG).
+ */
+CP_API cp_status cp_ulysses_permute_n(const void* const* srcs, void* const* dsts, int n_tensors, int degree,
+                               int B, int S, int H, int D, int direction, int elem_bytes, void* stream);
+
+/*
  * cp_ring_bounds - host-only helper: block bounds for a ring of n over S rows.
  *
  * Source: "Context parallelism", variants table: Ring Attention needs S divisible by

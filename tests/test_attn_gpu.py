@@ -130,3 +130,19 @@ def test_binding_checks_mirror_dispatcher():
     with pytest.raises(binding.CpError) as e:
         binding.attn_fwd(q96, k96, v96)
     assert e.value.status == binding.CP_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32], ids=["bf16", "fp32"])
+def test_output_only_16_byte_aligned(out_dtype):
+    """An output buffer aligned to 16 but not 32 bytes takes the 16-byte store path."""
+    B, H, Sq, Skv, D = 1, 2, 200, 300, 128
+    q, k, v = qkv(B, H, Sq, Skv, D, seed=17)
+    o_ref, lse_ref = oracle.attention(q, k, v, D ** -0.5)
+    n = B * Sq * H * D
+    shift = 16 // torch.tensor([], dtype=out_dtype).element_size()
+    buf = torch.full((n + shift,), float("nan"), dtype=out_dtype, device="cuda")
+    out = buf[shift:].view(B, Sq, H, D)
+    assert out.data_ptr() % 32 == 16
+    binding.attn_fwd(*cuda(q, k, v), out_dtype=out_dtype, out=out)
+    torch.cuda.synchronize()
+    assert_attn_close(out, None, o_ref, lse_ref, "16-byte aligned output")

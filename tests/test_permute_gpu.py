@@ -59,3 +59,21 @@ def test_ulysses_attention_bit_exact_vs_unsplit():
     o_seq = binding.ulysses_permute(o_h.view(P, B, S, H // P, D), P, 1)             # [P,B,S/P,H,D]
     o_back = o_seq.permute(1, 0, 2, 3, 4).reshape(B, S, H, D)
     assert torch.equal(o_back, o_full)
+
+
+def test_batched_permute_matches_single():
+    g = torch.Generator().manual_seed(5)
+    xs = [torch.randn(8, 1, 576, 24, 128, generator=g).bfloat16().cuda() for _ in range(3)]
+    ys = binding.ulysses_permute_n(xs, 8, 0)
+    for x, y in zip(xs, ys):
+        assert torch.equal(y, binding.ulysses_permute(x, 8, 0))
+    back = binding.ulysses_permute_n(ys, 8, 1)
+    for x, b in zip(xs, back):
+        assert torch.equal(x, b)
+
+
+def test_batched_permute_rejects_overlap():
+    x = torch.zeros(2, 1, 4, 4, 64, dtype=torch.bfloat16, device="cuda")
+    y = torch.zeros(2, 1, 8, 2, 64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(binding.CpError):
+        binding.ulysses_permute_n([x, x], 2, 0, dsts=[y, y])  # two destinations alias
