@@ -111,6 +111,23 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(mhz)}
 
 
+def reduce_max(value: float, device) -> float:
+    """Maximum of `value` over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, flop_per_step: float, total_ms: float, steps: int) -> float:
+    """Whole-job TFLOP/s: every rank runs `steps` steps of `flop_per_step`; time = slowest rank."""
+    return world * flop_per_step / (total_ms / steps * 1e-3) / 1e12
+
+
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -205,11 +222,7 @@ def run_ours(args):
     attn_ms = [e[1].elapsed_time(e[2]) for e in evs]
     merge_ms = [e[2].elapsed_time(e[3]) for e in evs]
     inv_ms = [e[3].elapsed_time(e[4]) for e in evs]
-    total_ms = sum(step_ms)
-    tot = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(tot, op=dist.ReduceOp.MAX)
-    total_ms = float(tot.item())
+    total_ms = reduce_max(sum(step_ms), dev)
 
     # Single-block attention (the FLUX ring-1 case) timed on its own.
     qd, kd, vd = (t.to(dev) for t in (q_h, k_h, v_h))
@@ -225,6 +238,22 @@ def run_ours(args):
         r1.append((a, b))
     torch.cuda.synchronize()
     ring1_ms = statistics.mean(a.elapsed_time(b) for a, b in r1[max(args.warmup, 3):])
+
+    # The ring with the LSE merge fused into the attention kernel (no partials, no merge
+    # pass), on the same head-sharded tensors as the step.
+    fo = torch.empty_like(o_h)
+    fl = torch.empty_like(lse_h)
+    view = lambda t: t.view(Bp, S, Hp, D)
+    rf = []
+    for i in range(max(args.warmup, 3) + 50):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        binding.ring_sim_fused(view(yq), view(yk), view(yv), bounds, scale=scale, out=fo, out_lse=fl)
+        b.record()
+        rf.append((a, b))
+    torch.cuda.synchronize()
+    fused_ms = statistics.mean(a.elapsed_time(b) for a, b in rf[max(args.warmup, 3):])
 
     # End to end through the public API with host buffers (pinned), per step:
     # H2D of the sequence-sharded Q/K/V, the hot path, D2H of O.
@@ -251,7 +280,7 @@ def run_ours(args):
     if rank == 0:
         peaks = load_peaks()
         step_mean = total_ms / args.steps
-        value = world * flop / (total_ms / args.steps * 1e-3) / 1e12
+        value = job_throughput(world, flop, total_ms, args.steps)
         attn_mean = statistics.mean(attn_ms)
         attn_tflops = flop / (attn_mean * 1e-3) / 1e12
         ring1_tflops = flop / (ring1_ms * 1e-3) / 1e12
@@ -300,6 +329,8 @@ def run_ours(args):
                 "attn_ring1_tflops": round(ring1_tflops, 2),
                 "attn_ring1_ms": round(ring1_ms, 4),
                 "attn_ring8_ms": round(attn_mean, 4),
+                "ring8_fused_ms": round(fused_ms, 4),
+                "ring8_fused_tflops": round(flop / (fused_ms * 1e-3) / 1e12, 2),
                 "attn_ring8_partial_bytes": part_bytes,
                 "merge_ms": round(statistics.mean(merge_ms), 4),
                 "merge_gbs": round(merge_bytes / (statistics.mean(merge_ms) * 1e-3) / 1e9, 1),

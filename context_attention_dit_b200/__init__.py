@@ -14,6 +14,7 @@ from .binding import (  # noqa: F401
     load,
     ring_bounds,
     ring_sim,
+    ring_sim_fused,
     ring_workspace_size,
     ring_workspace_views,
     status_string,
@@ -22,6 +23,6 @@ from .binding import (  # noqa: F401
 )
 
 __all__ = [
-    "CpError", "attn_fwd", "attn_fwd_blocks", "attn_merge", "last_device_status", "load", "ring_bounds", "ring_sim",
+    "CpError", "attn_fwd", "attn_fwd_blocks", "attn_merge", "last_device_status", "load", "ring_bounds", "ring_sim", "ring_sim_fused",
     "ring_workspace_size", "ring_workspace_views", "status_string", "ulysses_permute", "ulysses_permute_n",
 ]

@@ -32,8 +32,9 @@ CP_F32 = 1
 CP_MAX_CHUNKS = 64
 
 EXPORTS = (
-    "cp_attn_fwd", "cp_attn_fwd_blocks", "cp_attn_merge", "cp_ring_sim_workspace_size", "cp_ring_sim", "cp_ulysses_permute",
-    "cp_ulysses_permute_n", "cp_ring_bounds", "cp_last_device_status", "cp_status_string", "cp_version",
+    "cp_attn_fwd", "cp_attn_fwd_blocks", "cp_attn_merge", "cp_ring_sim_workspace_size", "cp_ring_sim",
+    "cp_ring_sim_fused", "cp_ring_sim_static", "cp_ulysses_permute", "cp_ulysses_permute_n", "cp_ring_bounds",
+    "cp_debug_set_fault", "cp_last_device_status", "cp_status_string", "cp_version",
 )
 
 _lib = None
@@ -61,11 +62,15 @@ def load() -> ctypes.CDLL:
     lib.cp_ring_sim_workspace_size.argtypes = [i, i, i, i, i]
     lib.cp_ring_sim_workspace_size.restype = sz
     lib.cp_ring_sim.argtypes = [vp, vp, vp, ip, i, vp, vp, i, i, i, i, i, f, i, vp, sz, vp]
+    lib.cp_ring_sim_fused.argtypes = [vp, vp, vp, ip, i, vp, vp, i, i, i, i, i, f, i, vp]
+    lib.cp_ring_sim_fused.restype = ctypes.c_int
     lib.cp_ring_sim_static.argtypes = [vp, vp, vp, ip, i, vp, vp, i, i, i, i, i, f, i, vp]
     lib.cp_ulysses_permute.argtypes = [vp, vp, i, i, i, i, i, i, i, vp]
     lib.cp_ulysses_permute_n.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), i, i, i, i, i, i, i, i, vp]
     lib.cp_ulysses_permute_n.restype = ctypes.c_int
     lib.cp_ring_bounds.argtypes = [i, i, i, ip]
+    lib.cp_debug_set_fault.argtypes = [i]
+    lib.cp_debug_set_fault.restype = ctypes.c_int
     lib.cp_last_device_status.argtypes = [vp]
     lib.cp_status_string.argtypes = [i]
     lib.cp_status_string.restype = ctypes.c_char_p
@@ -208,6 +213,26 @@ def ring_sim(q, k, v, chunk_bounds: Sequence[int], scale: Optional[float] = None
     return out, out_lse, workspace
 
 
+def ring_sim_fused(q, k, v, chunk_bounds: Sequence[int], scale: Optional[float] = None, out_dtype=torch.bfloat16,
+                   out=None, out_lse=None):
+    """Ring attention over K/V blocks with the LSE merge fused into the kernel; returns ``(out, lse)``."""
+    B, Sq, Skv, H, D = _check_qkv(q, k, v)
+    code = _out_code(out_dtype)
+    scale = float(D ** -0.5 if scale is None else scale)
+    n = len(chunk_bounds) - 1
+    if n < 1:
+        raise ValueError("chunk_bounds needs at least two entries")
+    bounds = (ctypes.c_int * (n + 1))(*[int(c) for c in chunk_bounds])
+    if out is None:
+        out = torch.empty((B, Sq, H, D), dtype=out_dtype, device=q.device)
+    if out_lse is None:
+        out_lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
+    st = load().cp_ring_sim_fused(_ptr(q), _ptr(k), _ptr(v), bounds, n, _ptr(out), _ptr(out_lse), B, H, Sq, Skv, D,
+                                  scale, code, ctypes.c_void_p(_stream(q)))
+    _check(st, "cp_ring_sim_fused")
+    return out, out_lse
+
+
 STATIC_SCRATCH_BYTES = 32 << 20
 
 
@@ -327,6 +352,11 @@ def ring_bounds(S: int, n: int, anything: bool = False):
     out = (ctypes.c_int * (n + 1))()
     _check(load().cp_ring_bounds(int(S), int(n), 1 if anything else 0, out), "cp_ring_bounds")
     return list(out)
+
+
+def debug_set_fault(mode: int):
+    """Test hook: mode 1 makes the next attention launch time out (see cpattn.h)."""
+    _check(load().cp_debug_set_fault(int(mode)), "cp_debug_set_fault")
 
 
 def last_device_status(stream=None) -> int:

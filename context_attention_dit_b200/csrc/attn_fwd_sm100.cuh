@@ -75,6 +75,9 @@ struct AttnParams {
   float* lse;                // block c at lse + c*lse_chunk_stride, [B][H][Sq]; may be null
   long long lse_chunk_stride;
   int* status;               // device status word
+  int fuse;                  // 1: one running softmax over all blocks, one merged output
+  int fault;                 // test hook: 1 = the producer never loads the CTA's first K tile
+  int first_c, last_c;       // first / last non-empty block (-1 if none)
   int bounds[kMaxChunks + 1];  // K/V row bounds of the blocks
 };
 
@@ -115,10 +118,15 @@ __device__ __forceinline__ UnitCoord decode_unit(int u, const AttnParams& p) {
 
 // One 128-key (or shorter) tile of K/V block c.
 struct Tile {
-  int c, j;     // block, tile within the block
-  int row0;     // first K/V row
-  int valid;    // keys of the block in this tile (1..128)
-  bool first, last;
+  int c, j;   // block, tile within the block
+  int row0;   // first K/V row
+  int info;   // bits 0-7: keys of the block in this tile (1..128); bit 8: last tile of its
+              // block (drives the tile walk); bits 9/10: first / last tile of a softmax
+              // segment (a block, or every block if fused)
+  __device__ __forceinline__ int valid() const { return info & 0xFF; }
+  __device__ __forceinline__ bool block_last() const { return (info >> 8) & 1; }
+  __device__ __forceinline__ bool first() const { return (info >> 9) & 1; }
+  __device__ __forceinline__ bool last() const { return (info >> 10) & 1; }
 };
 
 __device__ __forceinline__ int block_tiles(const AttnParams& p, int c) {
@@ -131,9 +139,12 @@ __device__ __forceinline__ Tile make_tile(const AttnParams& p, int c, int j) {
   t.j = j;
   const int len = p.bounds[c + 1] - p.bounds[c];
   t.row0 = p.bounds[c] + j * kBN;
-  t.valid = min(kBN, len - j * kBN);
-  t.first = (j == 0);
-  t.last = (j == (len + kBN - 1) / kBN - 1);
+  // first / last: the tile starts / ends a softmax segment (a block, or with p.fuse the
+  // whole run of blocks).
+  const int block_last = (j == (len + kBN - 1) / kBN - 1);
+  const int first = (j == 0) && (!p.fuse || c == p.first_c);
+  const int last = block_last && (!p.fuse || c == p.last_c);
+  t.info = min(kBN, len - j * kBN) | (block_last << 8) | (first << 9) | (last << 10);
   return t;
 }
 
@@ -148,7 +159,7 @@ __device__ __forceinline__ bool first_tile_from(const AttnParams& p, int c, Tile
 }
 
 __device__ __forceinline__ bool next_tile(const AttnParams& p, const Tile& cur, Tile& nxt) {
-  if (!cur.last) {
+  if (!cur.block_last()) {
     nxt = make_tile(p, cur.c, cur.j + 1);
     return true;
   }
@@ -198,11 +209,15 @@ __device__ __forceinline__ void attn_producer(const CUtensorMap* tm_q, const CUt
         const int st = kc_k % kStages;
         const uint32_t use = kc_k / kStages;
         if (use > 0 && !mbar_wait(bars + kKEmpty + st, (use - 1) & 1, abort_flag, p.status)) { ok = false; break; }
-        mbar_arrive_expect_tx(bars + kKFull + st, L::kTileBytes);
+        // Test hook (p.fault == 1): skip the CTA's first K tile, so that the consumer's
+        // bounded wait runs out and the kernel returns CP_ERR_TIMEOUT.
+        if (!(p.fault == 1 && kc_k == 0)) {
+          mbar_arrive_expect_tx(bars + kKFull + st, L::kTileBytes);
 #pragma unroll
-        for (int hf = 0; hf < D / 64; ++hf)
-          tma_load_4d(smem + L::kK + st * L::kTileBytes + hf * L::kHalfBytes, tm_k, bars + kKFull + st, hf * 64,
-                      uc.h, t.row0, uc.b);
+          for (int hf = 0; hf < D / 64; ++hf)
+            tma_load_4d(smem + L::kK + st * L::kTileBytes + hf * L::kHalfBytes, tm_k, bars + kKFull + st, hf * 64,
+                        uc.h, t.row0, uc.b);
+        }
         ++kc_k;
       }
       {
@@ -253,7 +268,7 @@ __device__ __forceinline__ void attn_mma(const AttnParams& p, uint8_t* smem, uin
     const uint32_t d_tmem = tmem + w * kBN;
     const uint32_t qbase = sQ + w * L::kTileBytes;
     const uint32_t kbase = sK + kst * L::kTileBytes;
-    const uint32_t idesc = t.valid > 64 ? kIdescQK128 : kIdescQK64;
+    const uint32_t idesc = t.valid() > 64 ? kIdescQK128 : kIdescQK64;
 #pragma unroll
     for (int k = 0; k < D / 16; ++k) {
       const uint32_t off = (k >> 2) * L::kHalfBytes + (k & 3) * 32;
@@ -267,10 +282,10 @@ __device__ __forceinline__ void attn_mma(const AttnParams& p, uint8_t* smem, uin
     const uint32_t a_tmem = tmem + w * kBN;
     const uint32_t o_tmem = tmem + 256 + w * 128;
     const uint32_t vbase = sV + vst * L::kTileBytes;
-    const int ksteps = t.valid > 64 ? kBN / 16 : 64 / 16;
+    const int ksteps = t.valid() > 64 ? kBN / 16 : 64 / 16;
     for (int k = 0; k < ksteps; ++k)
       tc_mma_ts(o_tmem, a_tmem + k * 8, sdesc_sw128(vbase + k * 2048, L::kHalfBytes, 1024), kIdescPV,
-                (!t.first || k > 0) ? 1u : 0u);
+                (!t.first() || k > 0) ? 1u : 0u);
   };
   auto wait_k = [&]() -> bool {
     if (!mbar_wait(bars + kKFull + (kc_k % kStages), (kc_k / kStages) & 1, abort_flag, p.status)) return false;
@@ -298,12 +313,12 @@ __device__ __forceinline__ void attn_mma(const AttnParams& p, uint8_t* smem, uin
 #pragma unroll
       for (int w = 0; w < kQTiles; ++w) {
         if (!mbar_wait(bars + kPReady + w, g & 1, abort_flag, p.status)) goto done;
-        if (cur.first && nch > 0) {
+        if (cur.first() && nch > 0) {
           if (!mbar_wait(bars + kOFree + w, (nch - 1) & 1, abort_flag, p.status)) goto done;
         }
         tc_fence_after();
         issue_pv(w, cur, vst);
-        if (cur.last) tc_commit(bars + kODone + w);
+        if (cur.last()) tc_commit(bars + kODone + w);
         if (more) {
           if (w == 0 && !wait_k()) goto done;
           issue_qk(w, nxt, kc_k % kStages);
@@ -316,7 +331,7 @@ __device__ __forceinline__ void attn_mma(const AttnParams& p, uint8_t* smem, uin
         ++kc_k;
       }
       ++g;
-      if (cur.last) ++nch;
+      if (cur.last()) ++nch;
       if (!more) break;
       cur = nxt;
       more = next_tile(p, cur, nxt);
@@ -486,29 +501,35 @@ __device__ __forceinline__ void attn_softmax(const AttnParams& p, uint8_t* smem,
   for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
     const UnitCoord uc = decode_unit(u, p);
     const int s_row = (uc.qp * kQTiles + w) * kBM + row;
+    float m = -INFINITY;  // running max of S*scale*log2e (possibly stale by < 8)
+    float l = 0.f;        // running sum of 2^(S*scale*log2e - m)
+    if (p.fuse && p.first_c < 0 && s_row < p.Sq) write_empty_row<D>(p, 0, uc, s_row);  // no keys at all
     for (int c = 0; c < p.n_chunks; ++c) {
       const int n_kv = block_tiles(p, c);
-      if (n_kv == 0) {  // no keys: O = 0, lse = -inf
-        if (s_row < p.Sq) write_empty_row<D>(p, c, uc, s_row);
+      if (n_kv == 0) {  // no keys: O = 0, lse = -inf (fused: the block simply adds nothing)
+        if (!p.fuse && s_row < p.Sq) write_empty_row<D>(p, c, uc, s_row);
         continue;
       }
-      float m = -INFINITY;  // running max of S*scale*log2e (possibly stale by < 8)
-      float l = 0.f;        // running sum of 2^(S*scale*log2e - m)
+      if (!p.fuse || c == p.first_c) {
+        m = -INFINITY;
+        l = 0.f;
+      }
       for (int j = 0; j < n_kv; ++j, ++g) {
         const Tile t = make_tile(p, c, j);
         if (!warp_wait(bars + kSFull + w, g & 1, abort_flag, p.status)) return;
         tc_fence_after();
-        if (t.valid == 128)
-          softmax_tile<D, 128, false>(ts, to, t.valid, t.first, sl2, m, l);
-        else if (t.valid > 64)
-          softmax_tile<D, 128, true>(ts, to, t.valid, t.first, sl2, m, l);
-        else if (t.valid == 64)
-          softmax_tile<D, 64, false>(ts, to, t.valid, t.first, sl2, m, l);
+        if (t.valid() == 128)
+          softmax_tile<D, 128, false>(ts, to, t.valid(), t.first(), sl2, m, l);
+        else if (t.valid() > 64)
+          softmax_tile<D, 128, true>(ts, to, t.valid(), t.first(), sl2, m, l);
+        else if (t.valid() == 64)
+          softmax_tile<D, 64, false>(ts, to, t.valid(), t.first(), sl2, m, l);
         else
-          softmax_tile<D, 64, true>(ts, to, t.valid, t.first, sl2, m, l);
+          softmax_tile<D, 64, true>(ts, to, t.valid(), t.first(), sl2, m, l);
         tc_fence_before();
         mbar_arrive(bars + kPReady + w);
       }
+      if (p.fuse && c != p.last_c) continue;  // the segment goes on with the next block
       // Hand (m, l) of this block to the epilogue warpgroup.  First wait until the epilogue
       // has finished the previous block (it releases O_w only after reading that block's
       // stats): without this wait, blocks of a single tile let this warpgroup run two
@@ -538,8 +559,10 @@ __device__ __forceinline__ void attn_epilogue(const AttnParams& p, uint8_t* smem
   if (p.tiles_per_unit == 0) return;
   for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
     const UnitCoord uc = decode_unit(u, p);
-    for (int c = 0; c < p.n_chunks; ++c) {
-      if (block_tiles(p, c) == 0) continue;
+    for (int c0 = 0; c0 < p.n_chunks; ++c0) {
+      if (block_tiles(p, c0) == 0) continue;
+      if (p.fuse && c0 != p.last_c) continue;  // one merged output per unit
+      const int c = p.fuse ? 0 : c0;             // output block index
 #pragma unroll 1
       for (int w = 0; w < kQTiles; ++w) {
         if (!warp_wait(bars + kStatReady + w, nch & 1, abort_flag, p.status)) return;

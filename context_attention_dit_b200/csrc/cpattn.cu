@@ -37,6 +37,7 @@ struct DeviceInfo {
 
 std::mutex g_mutex;
 DeviceInfo g_dev[kMaxDevices];
+int g_fault_next = 0;  // test hook consumed by the next attention launch
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -103,7 +104,7 @@ cp_status check_attn_args(const void* q, const void* k, const void* v, const voi
 // Launch the attention kernel over n_chunks K/V blocks given by `bounds` (host array).
 cp_status launch_attn(const void* q, const void* k, const void* v, const int* bounds, int n_chunks, void* out,
                       int out_f32, long long out_chunk_stride, float* lse, long long lse_chunk_stride, int B, int H,
-                      int Sq, int Skv, int D, float scale, cudaStream_t stream) {
+                      int Sq, int Skv, int D, float scale, cudaStream_t stream, int fuse = 0) {
   DeviceInfo* dev = nullptr;
   cp_status st = device_info(&dev);
   if (st != CP_OK) return st;
@@ -126,6 +127,18 @@ cp_status launch_attn(const void* q, const void* k, const void* v, const int* bo
   p.lse_chunk_stride = lse_chunk_stride;
   p.status = dev->status;
   for (int i = 0; i <= n_chunks; ++i) p.bounds[i] = bounds[i];
+  p.fuse = fuse;
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    p.fault = g_fault_next;
+    g_fault_next = 0;
+  }
+  p.first_c = p.last_c = -1;
+  for (int i = 0; i < n_chunks; ++i)
+    if (bounds[i + 1] > bounds[i]) {
+      if (p.first_c < 0) p.first_c = i;
+      p.last_c = i;
+    }
 
   CUtensorMap tq, tk, tv;
   // A map needs at least one row; with Skv == 0 every block is empty and K/V are never read.
@@ -164,35 +177,29 @@ cp_status launch_merge(const float* partials, const float* lses, int n, void* ou
   const long long rows = static_cast<long long>(B) * H * Sq;
   const long long part_stride = rows * D;
   const long long lse_stride = rows;
-  const long long blocks = (rows + kMergeThreads / 32 - 1) / (kMergeThreads / 32);
-  if (blocks >= (1LL << 31)) return CP_ERR_UNSUPPORTED;
-  const dim3 grid(static_cast<unsigned>(blocks));
+  // ST query positions per block (all heads), about 128 rows per block.
+  const int ST = H >= 128 ? 1 : (128 / H > 64 ? 64 : 128 / H);
+  const long long gx = (Sq + ST - 1) / ST;
+  if (B > 65535 || gx >= (1LL << 31)) return CP_ERR_UNSUPPORTED;
+  const size_t smem = static_cast<size_t>(n) * H * ST * sizeof(float);
+  if (smem > 48 * 1024) return CP_ERR_UNSUPPORTED;
+  const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(B));
   if (D == 128) {
     if (out_dtype == CP_BF16)
-      lse_merge_kernel<128, true><<<grid, kMergeThreads, 0, stream>>>(partials, lses, n, out, out_lse, H, Sq, rows,
-                                                                      part_stride, lse_stride);
+      lse_merge_kernel<128, true><<<grid, kMergeThreads, smem, stream>>>(partials, lses, n, out, out_lse, H, Sq, ST,
+                                                                         part_stride, lse_stride);
     else
-      lse_merge_kernel<128, false><<<grid, kMergeThreads, 0, stream>>>(partials, lses, n, out, out_lse, H, Sq, rows,
-                                                                       part_stride, lse_stride);
+      lse_merge_kernel<128, false><<<grid, kMergeThreads, smem, stream>>>(partials, lses, n, out, out_lse, H, Sq, ST,
+                                                                          part_stride, lse_stride);
   } else {
     if (out_dtype == CP_BF16)
-      lse_merge_kernel<64, true><<<grid, kMergeThreads, 0, stream>>>(partials, lses, n, out, out_lse, H, Sq, rows,
-                                                                     part_stride, lse_stride);
+      lse_merge_kernel<64, true><<<grid, kMergeThreads, smem, stream>>>(partials, lses, n, out, out_lse, H, Sq, ST,
+                                                                        part_stride, lse_stride);
     else
-      lse_merge_kernel<64, false><<<grid, kMergeThreads, 0, stream>>>(partials, lses, n, out, out_lse, H, Sq, rows,
-                                                                      part_stride, lse_stride);
+      lse_merge_kernel<64, false><<<grid, kMergeThreads, smem, stream>>>(partials, lses, n, out, out_lse, H, Sq, ST,
+                                                                         part_stride, lse_stride);
   }
   return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
-}
-
-cp_status check_bounds(const int* chunk_bounds, int n_chunks, int Skv) {
-  if (n_chunks < 1 || !chunk_bounds) return CP_ERR_INVALID_ARG;
-  if (n_chunks > CP_MAX_CHUNKS) return CP_ERR_UNSUPPORTED;
-  if (Skv < 0) return CP_ERR_INVALID_ARG;
-  if (chunk_bounds[0] != 0 || chunk_bounds[n_chunks] != Skv) return CP_ERR_INVALID_ARG;
-  for (int i = 0; i < n_chunks; ++i)
-    if (chunk_bounds[i] > chunk_bounds[i + 1]) return CP_ERR_INVALID_ARG;
-  return CP_OK;
 }
 
 inline size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -328,6 +335,17 @@ cp_status cp_ring_sim_static(const void* q, const void* k, const void* v, const 
                      need, stream);
 }
 
+cp_status cp_ring_sim_fused(const void* q, const void* k, const void* v, const int* chunk_bounds, int n_chunks,
+                            void* out, float* out_lse, int B, int H, int Sq, int Skv, int D, float scale,
+                            cp_dtype out_dtype, void* stream) {
+  cp_status st = check_bounds(chunk_bounds, n_chunks, Skv);
+  if (st != CP_OK) return st;
+  st = check_attn_args(q, k, v, out, out_lse, B, H, Sq, Skv, D, scale, out_dtype);
+  if (st != CP_OK || B == 0 || H == 0 || Sq == 0) return st;
+  return launch_attn(q, k, v, chunk_bounds, n_chunks, out, out_dtype == CP_F32 ? 1 : 0, 0, out_lse, 0, B, H, Sq, Skv,
+                     D, scale, static_cast<cudaStream_t>(stream), 1);
+}
+
 cp_status cp_ulysses_permute_n(const void* const* srcs, void* const* dsts, int n_tensors, int degree, int B, int S,
                                int H, int D, int direction, int elem_bytes, void* stream) {
   if (degree < 1 || B < 0 || S < 0 || H < 0 || D < 0) return CP_ERR_INVALID_ARG;
@@ -393,6 +411,13 @@ cp_status cp_ulysses_permute(const void* src, void* dst, int degree, int B, int 
   if (B == 0 || S == 0 || H == 0 || D == 0) return CP_OK;
   if (!src || !dst) return CP_ERR_INVALID_ARG;
   return cp_ulysses_permute_n(&src, &dst, 1, degree, B, S, H, D, direction, elem_bytes, stream);
+}
+
+cp_status cp_debug_set_fault(int mode) {
+  if (mode < 0 || mode > 1) return CP_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  g_fault_next = mode;
+  return CP_OK;
 }
 
 cp_status cp_ring_bounds(int S, int n, int anything, int* bounds_out) {

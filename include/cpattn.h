@@ -139,6 +139,22 @@ CP_API cp_status cp_ring_sim(const void* q, const void* k, const void* v, const 
                       int D, float scale, cp_dtype out_dtype, void* workspace, size_t ws_bytes,
                       void* stream);
 
+/*
+ * cp_ring_sim_fused - cp_ring_sim with the LSE merge fused into the attention kernel.
+ *
+ * Source: "Context parallelism", "Ring Attention" / "Ring Anything Attention": a GPU's
+ * queries meet the K/V blocks one after another and accumulate the result.  Here the
+ * running (max, sum, output) of each query row is carried in TMEM from one block to the
+ * next inside one launch, so no per-block partial is written and no merge pass runs; the
+ * result equals merging the per-block partials (up to fp32 rounding order).  Key tiles
+ * still end at block bounds, as in the unfused path.
+ * Arguments as cp_ring_sim without the workspace; allocates nothing.  Output and LSE as
+ * cp_attn_fwd; an all-empty split gives out = 0, lse = -inf.
+ */
+CP_API cp_status cp_ring_sim_fused(const void* q, const void* k, const void* v, const int* chunk_bounds,
+                            int n_chunks, void* out, float* out_lse, int B, int H, int Sq, int Skv,
+                            int D, float scale, cp_dtype out_dtype, void* stream);
+
 /* Size in bytes of the library's static device scratch used by cp_ring_sim_static. */
 #define CP_STATIC_SCRATCH_BYTES (32u << 20)
 
@@ -210,6 +226,18 @@ CP_API cp_status cp_ring_bounds(int S, int n, int anything, int* bounds_out);
  * CP_ERR_TIMEOUT if a kernel's bounded wait ran out since the last call.  Returns
  * CP_ERR_CUDA if the stream reported an error. */
 CP_API cp_status cp_last_device_status(void* stream);
+
+/*
+ * cp_debug_set_fault - test hook for the failure path (host only, no CUDA call).
+ *
+ * mode 1: the next attention launch (cp_attn_fwd, cp_attn_fwd_blocks, cp_ring_sim*) has its
+ * TMA producer skip one K tile.  The consumer's bounded wait then runs out (about one
+ * second), every warp leaves its loop, in-flight copies and MMAs are drained, TMEM is
+ * freed and the kernel returns; cp_last_device_status() then reports CP_ERR_TIMEOUT and the
+ * context stays usable.  The outputs of that launch are undefined.  mode 0 clears the hook.
+ * Nothing traps or faults.
+ */
+CP_API cp_status cp_debug_set_fault(int mode);
 
 /* Static string naming a status code. */
 CP_API const char* cp_status_string(cp_status s);

@@ -143,3 +143,46 @@ def test_ring_deterministic():
     outs = [binding.ring_sim(q, k, v, [0, 300, 301, 700], out_dtype=torch.float32)[:2] for _ in range(3)]
     for o, l in outs[1:]:
         assert torch.equal(o, outs[0][0]) and torch.equal(l, outs[0][1])
+
+
+@pytest.mark.parametrize(
+    "shape,bounds",
+    [
+        ((1, 2, 256, 256, 64), [0, 128, 256]),
+        ((2, 3, 300, 300, 128), [0, 100, 200, 300]),
+        ((1, 2, 200, 450, 128), [0, 0, 130, 130, 450]),     # empty blocks
+        ((1, 1, 129, 17, 64), [0, 5, 6, 17]),
+        ((1, 2, 150, 640, 128), [0, 640, 640]),
+    ],
+)
+def test_fused_ring_matches_oracle_and_unfused(shape, bounds):
+    """Fused merge (running softmax carried across blocks) == oracle ring == unfused ring."""
+    B, H, Sq, Skv, D = shape
+    q, k, v = qkv(B, H, Sq, Skv, D, seed=41)
+    scale = 1 / math.sqrt(D)
+    o_ref, lse_ref, _, _ = oracle.ring(q, k, v, scale, bounds)
+    dq, dk, dv = cuda(q, k, v)
+    o, lse = binding.ring_sim_fused(dq, dk, dv, bounds, scale=scale)
+    torch.cuda.synchronize()
+    assert binding.last_device_status() == 0
+    assert_attn_close(o, lse, o_ref, lse_ref, f"fused ring {bounds}")
+    o2, _, _ = binding.ring_sim(dq, dk, dv, bounds, scale=scale)
+    assert_split_close(o, o2, f"fused vs unfused {bounds}")
+
+
+def test_fused_ring_all_blocks_empty():
+    q, k, v = cuda(*qkv(1, 2, 130, 0, 128))
+    o, lse = binding.ring_sim_fused(q, k, v, [0, 0, 0])
+    torch.cuda.synchronize()
+    assert not o.float().abs().sum().item() and torch.isneginf(lse).all()
+
+
+def test_fused_flux_ring8_and_uneven():
+    w, (q, k, v) = workload_inputs("flux_1024_ring8_ulysses8")
+    o_ref, lse_ref = workload_oracle("flux_1024_ring1")
+    o, lse = binding.ring_sim_fused(*cuda(q, k, v), even_bounds(w.S, 8), scale=w.scale)
+    assert_attn_close(o, lse, o_ref, lse_ref, "fused flux ring-8")
+    w2, (q2, k2, v2) = workload_inputs("uneven_s4173_ring3")
+    o_ref2, lse_ref2 = workload_oracle("uneven_s4173_ring3")
+    o2, lse2 = binding.ring_sim_fused(*cuda(q2, k2, v2), bounds_from_sizes(w2.splits[1]), scale=w2.scale)
+    assert_attn_close(o2, lse2, o_ref2, lse_ref2, "fused uneven 1392/1391/1390")
