@@ -37,8 +37,10 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(s) <= t for s in sources() + [hdr, __file__])
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    if not force and up_to_date():
+def build(force: bool = False, verbose: bool = False, extra=(), out: str | None = None) -> str:
+    """Compile csrc/cpattn.cu into ``out`` (default: the in-tree libcpattn.so)."""
+    out = out or LIB
+    if out == LIB and not force and up_to_date():
         return LIB
     cmd = [
         nvcc_path(), "-O3", "-std=c++17", "-lineinfo",
@@ -47,15 +49,15 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
         "-cudart", "static",
         "-Xptxas", "-v" if verbose else "-O3",
         *extra,
-        "-o", LIB + ".tmp", os.path.join(CSRC, "cpattn.cu"),
+        "-o", out + ".tmp", os.path.join(CSRC, "cpattn.cu"),
     ]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if verbose or r.returncode != 0:
         sys.stderr.write(r.stdout + r.stderr)
     if r.returncode != 0:
         raise RuntimeError("nvcc failed building libcpattn.so:\n" + r.stderr[-4000:])
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(out + ".tmp", out)
+    return out
 
 
 if __name__ == "__main__":

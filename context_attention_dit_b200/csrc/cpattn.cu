@@ -202,6 +202,16 @@ cp_status launch_merge(const float* partials, const float* lses, int n, void* ou
   return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
 }
 
+cp_status check_bounds(const int* chunk_bounds, int n_chunks, int Skv) {
+  if (n_chunks < 1 || !chunk_bounds) return CP_ERR_INVALID_ARG;
+  if (n_chunks > CP_MAX_CHUNKS) return CP_ERR_UNSUPPORTED;
+  if (Skv < 0) return CP_ERR_INVALID_ARG;
+  if (chunk_bounds[0] != 0 || chunk_bounds[n_chunks] != Skv) return CP_ERR_INVALID_ARG;
+  for (int i = 0; i < n_chunks; ++i)
+    if (chunk_bounds[i] > chunk_bounds[i + 1]) return CP_ERR_INVALID_ARG;
+  return CP_OK;
+}
+
 inline size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 }  // namespace

@@ -35,6 +35,18 @@ def test_exported_symbols_in_dynamic_table():
     assert set(declared_functions()) <= exported
 
 
+def test_sources_compile_and_export_header(tmp_path):
+    """The current sources (not only the in-tree binary) build for sm_100a and export every
+    declared entry point."""
+    import subprocess
+
+    from context_attention_dit_b200 import build
+
+    out = build.build(out=str(tmp_path / "libcpattn_check.so"))
+    syms = subprocess.run(["nm", "-D", "--defined-only", out], capture_output=True, text=True).stdout
+    assert set(declared_functions()) <= set(re.findall(r"\b(cp_[a-z0-9_]+)\b", syms))
+
+
 def test_version_and_strings(lib):
     assert lib.cp_version() == 100
     for code in (0, -1, -2, -3, -4, -5, -6):
