@@ -7,31 +7,38 @@
 // per-block fp32 output + LSE follow ContextParallelConfig.convert_to_fp32 on the
 // "Parallelism" API page, so that ring blocks can be merged afterwards).
 //
-// Design (one CTA per SM, persistent over work units (b, h, pair of 128-row Q tiles);
-// each unit walks every K/V block and, inside a block, its 128-key tiles):
-//   warps 0-3   softmax warpgroup 0, Q tile 0 of the pair; thread t of warp w owns
-//   warps 4-7   softmax warpgroup 1, Q tile 1; its query row 32*(w%4)+t = TMEM lane.
-//               Per K/V tile: load the S row from TMEM, mask keys past the block end,
-//               update the running max m and sum l (base 2), write P = 2^(S*scale*log2e
-//               - m) as bf16 pairs into the first columns of the same S buffer.  After
-//               a block's last tile: hand the row's (m, l) to the epilogue warpgroup.
-//   warp 8      TMA producer: both Q tiles once per unit; K and V tiles (128 keys x D)
-//               through two 2-stage rings.  Warps 8-11 form the control warpgroup, which
-//               hands registers to the softmax warpgroups (setmaxnreg 88 / 184 / 56).
-//   warps 12-15 epilogue warpgroup: after a block's last P.V, read O_w from TMEM, release
-//               it for the next block, write O/l (fp32 partial or final bf16/fp32) and lse.
-//   warp 9      TMEM owner (512 columns) and MMA issuer (one thread), in the order
-//               QK0(t) QK1(t) | PV0(t) QK0(t+1) PV1(t) QK1(t+1) | ...
-//               S_w = Q_w K^T: SS form, both operands K-major and 128B-swizzled;
-//               O_w += P_w V: TS form, P_w read from TMEM, V MN-major in shared memory.
-//               Because QK_w(t+1) is issued after PV_w(t), the commit that signals "S_w
-//               full" also certifies that O_w holds every earlier P.V product.
-// TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [384,384+D).
-// A tile whose block has at most 64 keys left runs N = 64 (QK) and K = 64 (PV) MMAs and
-// a 64-column softmax.
-// The running max is updated lazily: O_w is rescaled in TMEM only when a row's max grows
-// by more than 8 (a factor 256); otherwise the stale max stays, which is exact because O
-// and l share it and 2^8 cannot overflow fp32 or bf16.
+// Design (one CTA per SM, persistent over work units (b, h, 128-row Q tile); each unit
+// walks every K/V block and, inside a block, its 128-key tiles):
+//   warps 0-3   softmax warpgroup 0: keys 0-63 of every K/V tile;
+//   warps 4-7   softmax warpgroup 1: keys 64-127.  Thread t of warp w owns query row
+//               32*(w%4)+t (= TMEM lane) and keeps its own running max m_k, sum l_k and
+//               accumulator O_k over its half k of the keys.  Per tile it loads its 64 S
+//               columns from TMEM, masks keys past the block end, updates m_k (lazily)
+//               and l_k, and stores P = 2^(S*scale*log2e - m_k) as bf16 over the first
+//               32 of those columns.  At a segment's end it hands (m_k, l_k) over.
+//   warp 8      TMA producer of Q (two slots, so the next unit's tile arrives early) and
+//               K (two stages).
+//   warp 10     TMA producer of V (two stages).
+//   warp 9      TMEM owner (512 columns) and QK issuer (one thread):
+//               S(t) = Q K(t)^T        SS form, into S buffer t%2, as soon as K(t) is
+//                                      loaded and PV(t-2) has consumed that buffer;
+//   warp 11     P.V issuer (one thread):
+//               O_k += P_k(t) V_k(t)   TS form (P from TMEM), once both warpgroups have
+//                                      stored P(t); V_k = rows 64k..64k+63 of V.
+//               The next S is computed while the softmax works on this tile, and each
+//               issuer's bookkeeping overlaps the other's MMAs.
+//   warps 12-15 epilogue warpgroup: after a segment's last P.V, merge the two halves,
+//               m = max(m_0, m_1), w_k = 2^(m_k - m),
+//               O = (w_0 O_0 + w_1 O_1) / (w_0 l_0 + w_1 l_1),
+//               lse = ln 2 * (m + log2(w_0 l_0 + w_1 l_1)),
+//               release O and write O (fp32 partial, or bf16/fp32) and lse.
+// A segment is one K/V block, or every block with p.fuse (cp_ring_sim_fused).
+// TMEM columns: S buffers [0,128) and [128,256) (P_k over columns 64k .. 64k+31 of its
+// buffer), O_0 [256,256+D), O_1 [384,384+D).
+// A tile with at most 64 keys runs an N = 64 QK and no P.V for half 1.
+// Lazy max: O_k is rescaled in TMEM only when a row's max grows by more than 8 (a factor
+// 256); otherwise the stale max stays, which is exact because O_k and l_k share it and
+// 2^8 cannot overflow fp32 or bf16.
 // Every mbarrier wait is bounded (see ptx_sm100.cuh); on a timeout every role leaves its
 // loop, in-flight TMA loads and MMAs are drained, TMEM is freed and the kernel returns
 // with CP_ERR_TIMEOUT recorded in the device status word.
@@ -43,29 +50,40 @@
 
 namespace cpattn {
 
-constexpr int kBM = 128;           // query rows per Q tile (TMEM lanes)
-constexpr int kQTiles = 2;         // Q tiles per work unit, one softmax warpgroup each
+constexpr int kBM = 128;           // query rows per work unit (TMEM lanes)
 constexpr int kBN = 128;           // keys per K/V tile
-constexpr int kStages = 2;         // stages of each of the K and V rings
+constexpr int kHalfN = 64;         // keys per softmax warpgroup and tile
+constexpr int kStages = 2;         // Q slots, K stages, V stages
 constexpr int kAttnThreads = 512;  // 16 warps: 2 softmax, 1 control, 1 epilogue warpgroup
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kProducerWarp = 8;   // Q and K loads
+constexpr int kMmaWarp = 9;       // TMEM owner, QK issuer
+constexpr int kVProducerWarp = 10; // V loads
+constexpr int kPvWarp = 11;        // P.V issuer
 constexpr int kEpilogueWarp0 = 12;
-// Registers per thread after the split (launch: 128 = 65536 / 512).
-// 256 * kSoftmaxRegs + 128 * kControlRegs + 128 * kEpilogueRegs = 512 * 128.
-constexpr int kSoftmaxRegs = 184;
-constexpr int kControlRegs = 88;
-constexpr int kEpilogueRegs = 56;
+// setmaxnreg split of the 128 x 512 launch budget: softmax (8 warps), control (warps 8-11),
+// epilogue (warps 12-15).
+constexpr int kSoftmaxRegs = 152;
+constexpr int kControlRegs = 96;
+constexpr int kEpilogueRegs = 112;
 static_assert(2 * kSoftmaxRegs + kControlRegs + kEpilogueRegs == 4 * 128, "register split must use the launch budget");
 constexpr int kTmemCols = 512;
+constexpr int kTmemO = 256;        // first O column; O_k at kTmemO + 128 k
 constexpr int kMaxChunks = 64;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// 2^x on the FMA pipe for one pair in kEmuEvery of a tile without masked keys (0: off):
+// n = rint(x) by the 1.5*2^23 shift, f = x - n in [-1/2, 1/2], 2^f by a degree-3 minimax
+// polynomial (relative error 7.5e-5, fitted for this kernel), 2^n added to the exponent.
+constexpr int kEmuEvery = 4;
+constexpr float kExp2C0 = 0.9999280571937561f;
+constexpr float kExp2C1 = 0.6932608485221863f;
+constexpr float kExp2C2 = 0.24261115491390228f;
+constexpr float kExp2C3 = 0.05517221987247467f;
 
 struct AttnParams {
   int B, H, Sq;
   int n_chunks;
-  int n_qp;                  // ceil(Sq / (kQTiles * kBM)) Q-tile pairs
-  int n_units;               // B * H * n_qp
+  int n_qt;                  // ceil(Sq / kBM) Q tiles
+  int n_units;               // B * H * n_qt
   int tiles_per_unit;        // sum over blocks of ceil(len / kBN)
   float scale_log2;          // scale * log2(e)
   void* out;                 // block c at out + c*out_chunk_stride elements, [B][Sq][H][D]
@@ -85,36 +103,45 @@ template <int D>
 struct AttnSmem {
   static constexpr int kHalfBytes = kBM * 64 * 2;  // 128 rows x 64 bf16: one 128B-swizzled box
   static constexpr int kTileBytes = kBM * D * 2;   // 128 rows x D bf16
-  static constexpr int kQ = 0;                     // kQTiles Q tiles
-  static constexpr int kK = kQ + kQTiles * kTileBytes;
-  static constexpr int kV = kK + kStages * kTileBytes;
-  static constexpr int kStat = kV + kStages * kTileBytes;  // float2 [kQTiles][2][kBM]: (m, l) per row
-  static constexpr int kBar = kStat + kQTiles * 2 * kBM * 8;
+  static constexpr int kQ = 0;                           // kStages Q slots
+  static constexpr int kK = kQ + kStages * kTileBytes;   // kStages K stages
+  static constexpr int kV = kK + kStages * kTileBytes;   // kStages V stages
+  static constexpr int kStat = kV + kStages * kTileBytes;  // float2 [2 halves][2 parities][kBM]: (m, l)
+  static constexpr int kBar = kStat + 2 * 2 * kBM * 8;
   static constexpr int kNumBars = 21;
   static constexpr int kUsed = kBar + kNumBars * 8 + 16;
-  // More than half an SM's shared memory: exactly one CTA (owning all 512 TMEM
-  // columns) is resident per SM.
+  // Request enough that at most one CTA fits per SM (the kernel allocates all 512 TMEM
+  // columns), plus 1 KB for aligning the base to the 128B-swizzle atom.
   static constexpr int kRequest = (kUsed + 1024) > 120 * 1024 ? (kUsed + 1024) : 120 * 1024;
 };
 
-// Barrier indices.
+// Barrier indices.  Tile t uses K stage, V stage and S buffer t % 2 (kStages = 2), so one
+// commit per tile and issuer serves every consumer of that slot:
+//   qk_done[t%2]  after S(t) = Q K(t)^T: S(t) is ready (softmax), K stage t%2 is free (K
+//                 producer);
+//   pv_done[t%2]  after O += P(t) V(t): V stage t%2 is free (V producer), S buffer t%2 is
+//                 free for QK(t+2), O holds every product up to tile t (softmax rescale).
+// p_ready is [S buffer][half].
 enum : int {
-  kQFull = 0, kQEmpty = 1, kKFull = 2, kKEmpty = 4, kVFull = 6, kVEmpty = 8,
-  kSFull = 10, kPReady = 12, kODone = 14, kOFree = 16, kStatReady = 18, kDrain = 20
+  kQFull = 0, kQEmpty = 2, kKFull = 4, kVFull = 6, kQkDone = 8, kPvDone = 10, kPReady = 12,
+  kODone = 16, kOFree = 17, kStatReady = 18, kDrain = 19, kDrainPV = 20
 };
 
 struct UnitCoord {
-  int b, h, qp;
+  int b, h, qt;
 };
 
 __device__ __forceinline__ UnitCoord decode_unit(int u, const AttnParams& p) {
   UnitCoord r;
-  r.qp = u % p.n_qp;
-  const int bh = u / p.n_qp;
+  r.qt = u % p.n_qt;
+  const int bh = u / p.n_qt;
   r.h = bh % p.H;
   r.b = bh / p.H;
   return r;
 }
+
+// Keys of a tile with `valid` keys that fall in half k (0..64).
+__device__ __forceinline__ int half_valid(int valid, int k) { return min(kHalfN, max(0, valid - k * kHalfN)); }
 
 // One 128-key (or shorter) tile of K/V block c.
 struct Tile {
@@ -172,6 +199,21 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, ok);
 }
 
+// Named barriers (id 0 is __syncthreads): one per softmax warpgroup and the epilogue.
+constexpr int kBarSoftmax0 = 1;
+constexpr int kBarEpilogue = 3;
+
+// A 128-thread warpgroup waits for `bar`: only its first warp polls (fewer mbarrier polls
+// in the MIO queue), the others park at named barrier `id`.  `alive` carries an earlier
+// failure of this thread into the decision, so that every warp of the group leaves
+// together: a named barrier that one warp never reaches would never complete.
+__device__ __forceinline__ bool group_wait(uint64_t* bar, uint32_t parity, int id, bool alive,
+                                           volatile int* abort_flag, int* status, uint32_t sleep_ns = 0) {
+  bool ok = alive;
+  if ((threadIdx.x & 127) < 32 && ok) ok = mbar_wait(bar, parity, abort_flag, status, sleep_ns);
+  return bar_and(id, 128, ok);
+}
+
 // Wait bounded by time only (used to drain in-flight work after an abort).
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   const long long t0 = clock64();
@@ -180,162 +222,138 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-// ------------------------------------------------------------------------------- producer
+// ------------------------------------------------------------------------------- producers
 
+// Warp 8, lane 0: the Q tile of every unit (two slots) and one K tile per K/V tile.
 template <int D>
-__device__ __forceinline__ void attn_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
-                                              const CUtensorMap* tm_v, const AttnParams& p, uint8_t* smem,
-                                              uint64_t* bars, volatile int* abort_flag) {
+__device__ __forceinline__ void attn_producer_qk(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
+                                                 const AttnParams& p, uint8_t* smem, uint64_t* bars,
+                                                 volatile int* abort_flag) {
   using L = AttnSmem<D>;
   if (p.tiles_per_unit == 0) return;
-  uint32_t kc_k = 0, kc_v = 0;  // tiles issued into the K and V rings
-  uint32_t n_q = 0;             // Q pairs issued
+  uint32_t kc = 0;   // K tiles issued
+  uint32_t n_q = 0;  // Q tiles issued
   bool ok = true;
   for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
     const UnitCoord uc = decode_unit(u, p);
-    if (n_q > 0 && !mbar_wait(bars + kQEmpty, (n_q - 1) & 1, abort_flag, p.status)) break;
-    mbar_arrive_expect_tx(bars + kQFull, kQTiles * L::kTileBytes);
-#pragma unroll
-    for (int w = 0; w < kQTiles; ++w)
+    {
+      const int qs = n_q % kStages;
+      const uint32_t use = n_q / kStages;
+      if (use > 0 && !mbar_wait(bars + kQEmpty + qs, (use - 1) & 1, abort_flag, p.status, 32)) break;
+      mbar_arrive_expect_tx(bars + kQFull + qs, L::kTileBytes);
 #pragma unroll
       for (int hf = 0; hf < D / 64; ++hf)
-        tma_load_4d(smem + L::kQ + w * L::kTileBytes + hf * L::kHalfBytes, tm_q, bars + kQFull, hf * 64, uc.h,
-                    (uc.qp * kQTiles + w) * kBM, uc.b);
-    ++n_q;
+        tma_load_4d(smem + L::kQ + qs * L::kTileBytes + hf * L::kHalfBytes, tm_q, bars + kQFull + qs, hf * 64, uc.h,
+                    uc.qt * kBM, uc.b);
+      ++n_q;
+    }
     Tile t;
     bool have = first_tile_from(p, 0, t);
     while (have) {
-      {
-        const int st = kc_k % kStages;
-        const uint32_t use = kc_k / kStages;
-        if (use > 0 && !mbar_wait(bars + kKEmpty + st, (use - 1) & 1, abort_flag, p.status)) { ok = false; break; }
-        // Test hook (p.fault == 1): skip the CTA's first K tile, so that the consumer's
-        // bounded wait runs out and the kernel returns CP_ERR_TIMEOUT.
-        if (!(p.fault == 1 && kc_k == 0)) {
-          mbar_arrive_expect_tx(bars + kKFull + st, L::kTileBytes);
-#pragma unroll
-          for (int hf = 0; hf < D / 64; ++hf)
-            tma_load_4d(smem + L::kK + st * L::kTileBytes + hf * L::kHalfBytes, tm_k, bars + kKFull + st, hf * 64,
-                        uc.h, t.row0, uc.b);
-        }
-        ++kc_k;
-      }
-      {
-        const int st = kc_v % kStages;
-        const uint32_t use = kc_v / kStages;
-        if (use > 0 && !mbar_wait(bars + kVEmpty + st, (use - 1) & 1, abort_flag, p.status)) { ok = false; break; }
-        mbar_arrive_expect_tx(bars + kVFull + st, L::kTileBytes);
+      const int st = kc % kStages;
+      const uint32_t use = kc / kStages;
+      if (use > 0 && !mbar_wait(bars + kQkDone + st, (use - 1) & 1, abort_flag, p.status, 32)) { ok = false; break; }
+      // Test hook (p.fault == 1): skip the CTA's first K tile, so that the consumer's
+      // bounded wait runs out and the kernel returns CP_ERR_TIMEOUT.
+      if (!(p.fault == 1 && kc == 0)) {
+        mbar_arrive_expect_tx(bars + kKFull + st, L::kTileBytes);
 #pragma unroll
         for (int hf = 0; hf < D / 64; ++hf)
-          tma_load_4d(smem + L::kV + st * L::kTileBytes + hf * L::kHalfBytes, tm_v, bars + kVFull + st, hf * 64,
+          tma_load_4d(smem + L::kK + st * L::kTileBytes + hf * L::kHalfBytes, tm_k, bars + kKFull + st, hf * 64,
                       uc.h, t.row0, uc.b);
-        ++kc_v;
       }
+      ++kc;
       have = next_tile(p, t, t);
     }
   }
   // Drain: every issued load lands before the CTA may exit (normal path: already done).
-  if (n_q > 0) drain_wait(bars + kQFull, (n_q - 1) & 1);
   for (int st = 0; st < kStages; ++st) {
-    const uint32_t uk = kc_k / kStages + (st < static_cast<int>(kc_k % kStages) ? 1u : 0u);
-    const uint32_t uv = kc_v / kStages + (st < static_cast<int>(kc_v % kStages) ? 1u : 0u);
+    const uint32_t uq = n_q / kStages + (st < static_cast<int>(n_q % kStages) ? 1u : 0u);
+    const uint32_t uk = kc / kStages + (st < static_cast<int>(kc % kStages) ? 1u : 0u);
+    if (uq > 0) drain_wait(bars + kQFull + st, (uq - 1) & 1);
     if (uk > 0) drain_wait(bars + kKFull + st, (uk - 1) & 1);
+  }
+}
+
+// Warp 10, lane 0: one V tile per K/V tile.
+template <int D>
+__device__ __forceinline__ void attn_producer_v(const CUtensorMap* tm_v, const AttnParams& p, uint8_t* smem,
+                                                uint64_t* bars, volatile int* abort_flag) {
+  using L = AttnSmem<D>;
+  if (p.tiles_per_unit == 0) return;
+  uint32_t vc = 0;  // V tiles issued
+  bool ok = true;
+  for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+    const UnitCoord uc = decode_unit(u, p);
+    Tile t;
+    bool have = first_tile_from(p, 0, t);
+    while (have) {
+      const int st = vc % kStages;
+      const uint32_t use = vc / kStages;
+      if (use > 0 && !mbar_wait(bars + kPvDone + st, (use - 1) & 1, abort_flag, p.status, 32)) { ok = false; break; }
+      mbar_arrive_expect_tx(bars + kVFull + st, L::kTileBytes);
+#pragma unroll
+      for (int hf = 0; hf < D / 64; ++hf)
+        tma_load_4d(smem + L::kV + st * L::kTileBytes + hf * L::kHalfBytes, tm_v, bars + kVFull + st, hf * 64, uc.h,
+                    t.row0, uc.b);
+      ++vc;
+      have = next_tile(p, t, t);
+    }
+  }
+  for (int st = 0; st < kStages; ++st) {
+    const uint32_t uv = vc / kStages + (st < static_cast<int>(vc % kStages) ? 1u : 0u);
     if (uv > 0) drain_wait(bars + kVFull + st, (uv - 1) & 1);
   }
 }
 
 // ------------------------------------------------------------------------------- MMA issuer
 
+// Warp 9, lane 0: S(t) = Q K(t)^T for every K/V tile t of the CTA (all its units), into
+// S buffer t%2: D/16 k-steps of 16; step k sits in the 64-column half k/4 at byte 32*(k%4)
+// (128B-swizzled K-major, 8-row groups 1 KB apart).  Buffer t%2 held P(t-2), so QK(t)
+// waits for pv_done of tile t-2: MMAs of different threads are not ordered with each
+// other.
 template <int D>
-__device__ __forceinline__ void attn_mma(const AttnParams& p, uint8_t* smem, uint64_t* bars, uint32_t tmem,
-                                         volatile int* abort_flag) {
+__device__ __forceinline__ void attn_mma_qk(const AttnParams& p, uint8_t* smem, uint64_t* bars, uint32_t tmem,
+                                            volatile int* abort_flag) {
   using L = AttnSmem<D>;
   if (p.tiles_per_unit == 0) return;
   constexpr uint32_t kIdescQK128 = idesc_bf16_f32(kBM, 128, 0);
   constexpr uint32_t kIdescQK64 = idesc_bf16_f32(kBM, 64, 0);
-  constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, D, 1);
   const uint32_t sQ = smem_u32(smem + L::kQ);
   const uint32_t sK = smem_u32(smem + L::kK);
-  const uint32_t sV = smem_u32(smem + L::kV);
-
-  uint32_t kc_k = 0, kc_v = 0;  // K/V ring positions consumed
-  uint32_t g = 0;               // tiles processed (S_w / P_w phase)
-  uint32_t nch = 0;             // non-empty blocks finished (O_w phase)
-  uint32_t n_q = 0;             // units started (Q phase)
-
-  // S_w = Q_w K^T: D/16 k-steps of 16; step k sits in 64-column half k/4 at byte 32*(k%4).
-  auto issue_qk = [&](int w, const Tile& t, int kst) {
-    const uint32_t d_tmem = tmem + w * kBN;
-    const uint32_t qbase = sQ + w * L::kTileBytes;
-    const uint32_t kbase = sK + kst * L::kTileBytes;
-    const uint32_t idesc = t.valid() > 64 ? kIdescQK128 : kIdescQK64;
-#pragma unroll
-    for (int k = 0; k < D / 16; ++k) {
-      const uint32_t off = (k >> 2) * L::kHalfBytes + (k & 3) * 32;
-      tc_mma_ss(d_tmem, sdesc_sw128(qbase + off, 16, 1024), sdesc_sw128(kbase + off, 16, 1024), idesc, k > 0);
-    }
-    tc_commit(bars + kSFull + w);
-  };
-  // O_w (+)= P_w V: P_w (bf16 pairs) in the S_w columns; V MN-major, 16 keys per k-step
-  // = 2048 bytes; the two 64-wide D halves are 16 KB apart (leading byte offset).
-  auto issue_pv = [&](int w, const Tile& t, int vst) {
-    const uint32_t a_tmem = tmem + w * kBN;
-    const uint32_t o_tmem = tmem + 256 + w * 128;
-    const uint32_t vbase = sV + vst * L::kTileBytes;
-    const int ksteps = t.valid() > 64 ? kBN / 16 : 64 / 16;
-    for (int k = 0; k < ksteps; ++k)
-      tc_mma_ts(o_tmem, a_tmem + k * 8, sdesc_sw128(vbase + k * 2048, L::kHalfBytes, 1024), kIdescPV,
-                (!t.first() || k > 0) ? 1u : 0u);
-  };
-  auto wait_k = [&]() -> bool {
-    if (!mbar_wait(bars + kKFull + (kc_k % kStages), (kc_k / kStages) & 1, abort_flag, p.status)) return false;
-    tc_fence_after();
-    return true;
-  };
-
+  uint32_t kc = 0;   // K tiles consumed
+  uint32_t g = 0;    // tiles whose QK has been issued
+  uint32_t n_q = 0;  // units started (Q slot use)
   for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
-    if (!mbar_wait(bars + kQFull, n_q & 1, abort_flag, p.status)) goto done;
-    tc_fence_after();
+    const int qs = n_q % kStages;
+    if (!mbar_wait(bars + kQFull + qs, (n_q / kStages) & 1, abort_flag, p.status)) goto done;
     ++n_q;
-    Tile cur, nxt;
-    first_tile_from(p, 0, cur);
-    // Prologue: S for the unit's first tile, both Q tiles.
-    if (!wait_k()) goto done;
-    issue_qk(0, cur, kc_k % kStages);
-    issue_qk(1, cur, kc_k % kStages);
-    tc_commit(bars + kKEmpty + (kc_k % kStages));
-    ++kc_k;
-    bool more = next_tile(p, cur, nxt);
-    if (!more) tc_commit(bars + kQEmpty);
-    while (true) {
-      const int vst = kc_v % kStages;
-      if (!mbar_wait(bars + kVFull + vst, (kc_v / kStages) & 1, abort_flag, p.status)) goto done;
+    const uint64_t qd = sdesc_sw128(sQ + qs * L::kTileBytes, 16, 1024);
+    Tile t;
+    bool have = first_tile_from(p, 0, t);
+    while (have) {
+      Tile nxt;
+      const bool more = next_tile(p, t, nxt);
+      const int kst = kc % kStages;
+      const int sb = g & 1;
+      if (g >= 2 && !mbar_wait(bars + kPvDone + sb, ((g >> 1) - 1) & 1, abort_flag, p.status)) goto done;
+      if (!mbar_wait(bars + kKFull + kst, (kc / kStages) & 1, abort_flag, p.status)) goto done;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem + sb * kBN;
+      const uint64_t kd = sdesc_sw128(sK + kst * L::kTileBytes, 16, 1024);
+      const uint32_t idesc = t.valid() > kHalfN ? kIdescQK128 : kIdescQK64;
 #pragma unroll
-      for (int w = 0; w < kQTiles; ++w) {
-        if (!mbar_wait(bars + kPReady + w, g & 1, abort_flag, p.status)) goto done;
-        if (cur.first() && nch > 0) {
-          if (!mbar_wait(bars + kOFree + w, (nch - 1) & 1, abort_flag, p.status)) goto done;
-        }
-        tc_fence_after();
-        issue_pv(w, cur, vst);
-        if (cur.last()) tc_commit(bars + kODone + w);
-        if (more) {
-          if (w == 0 && !wait_k()) goto done;
-          issue_qk(w, nxt, kc_k % kStages);
-        }
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t off = ((k >> 2) * L::kHalfBytes + (k & 3) * 32) >> 4;  // descriptor address units
+        tc_mma_ss(d_tmem, qd + off, kd + off, idesc, k > 0);
       }
-      tc_commit(bars + kVEmpty + vst);
-      ++kc_v;
-      if (more) {
-        tc_commit(bars + kKEmpty + (kc_k % kStages));
-        ++kc_k;
-      }
+      tc_commit(bars + kQkDone + sb);  // kst == sb
+      if (!more) tc_commit(bars + kQEmpty + qs);  // the unit's last QK: its Q slot frees
+      ++kc;
       ++g;
-      if (cur.last()) ++nch;
-      if (!more) break;
-      cur = nxt;
-      more = next_tile(p, cur, nxt);
-      if (!more) tc_commit(bars + kQEmpty);  // the unit's last QK has been issued
+      t = nxt;
+      have = more;
     }
   }
 done:
@@ -344,30 +362,89 @@ done:
   drain_wait(bars + kDrain, 0);
 }
 
+// Warp 11, lane 0: O_k (+)= P_k(t) V_k(t) once both softmax warpgroups have stored P(t).
+// P_k = 64 keys as bf16 pairs in 32 columns of S buffer t%2; V MN-major, 16 keys per
+// k-step = 2048 bytes, the two 64-wide D halves 16 KB apart (leading byte offset).
+template <int D>
+__device__ __forceinline__ void attn_mma_pv(const AttnParams& p, uint8_t* smem, uint64_t* bars, uint32_t tmem,
+                                            volatile int* abort_flag) {
+  using L = AttnSmem<D>;
+  if (p.tiles_per_unit == 0) return;
+  constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, D, 1);
+  const uint32_t sV = smem_u32(smem + L::kV);
+  uint32_t vc = 0;    // V tiles consumed
+  uint32_t gp = 0;    // tiles whose P.V has been issued
+  uint32_t nch = 0;   // segments finished (O phase)
+  bool init0 = false, init1 = false;  // O_k already written in the current segment
+  for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+    Tile t;
+    bool have = first_tile_from(p, 0, t);
+    while (have) {
+      const int vst = vc % kStages;
+      const int sb = gp & 1;
+      const uint32_t ppar = (gp >> 1) & 1;
+      if (t.first()) init0 = init1 = false;
+      if (!mbar_wait(bars + kVFull + vst, (vc / kStages) & 1, abort_flag, p.status)) goto done;
+      if (!mbar_wait(bars + kPReady + sb * 2, ppar, abort_flag, p.status)) goto done;
+      if (!mbar_wait(bars + kPReady + sb * 2 + 1, ppar, abort_flag, p.status)) goto done;
+      if (t.first() && nch > 0 && !mbar_wait(bars + kOFree, (nch - 1) & 1, abort_flag, p.status)) goto done;
+      tc_fence_after();
+      const uint64_t vd = sdesc_sw128(sV + vst * L::kTileBytes, L::kHalfBytes, 1024);
+      const uint32_t a0 = tmem + sb * kBN;
+      {
+        const uint32_t acc = init0 ? 1u : 0u;
+#pragma unroll
+        for (int ks = 0; ks < kHalfN / 16; ++ks)
+          tc_mma_ts(tmem + kTmemO, a0 + ks * 8, vd + ks * (2048 >> 4), kIdescPV, acc | (ks > 0 ? 1u : 0u));
+        init0 = true;
+      }
+      if (t.valid() > kHalfN) {
+        const uint32_t acc = init1 ? 1u : 0u;
+#pragma unroll
+        for (int ks = 0; ks < kHalfN / 16; ++ks)
+          tc_mma_ts(tmem + kTmemO + 128, a0 + kHalfN + ks * 8, vd + (4 + ks) * (2048 >> 4), kIdescPV,
+                    acc | (ks > 0 ? 1u : 0u));
+        init1 = true;
+      }
+      tc_commit(bars + kPvDone + sb);  // vst == sb
+      if (t.last()) {
+        tc_commit(bars + kODone);
+        ++nch;
+      }
+      ++vc;
+      ++gp;
+      have = next_tile(p, t, t);
+    }
+  }
+done:
+  tc_commit(bars + kDrainPV);
+  drain_wait(bars + kDrainPV, 0);
+}
+
 // ------------------------------------------------------------------------------- softmax
 
-// Softmax of one tile of NC (128 or 64) columns for this thread's row, in one pass over
-// TMEM: the whole S row is loaded into registers (one round trip), keys at or past
-// `valid` are masked when MASK (only a block's last tile), then the row max, the lazy
-// max update, and P = 2^(S*scale*log2e - m) with packed fp32x2 FMAs, MUFU ex2 and packed
-// sums.  On return P is stored as bf16 pairs in columns [0, NC/2) of the S buffer (the
-// whole row is already in registers, so the overwrite is safe) and l/m are updated.
-template <int D, int NC, bool MASK>
-__device__ __forceinline__ void softmax_tile(uint32_t ts, uint32_t to, int valid, bool first, float sl2, float& m,
-                                             float& l) {
-  uint32_t r[NC];
-  if (NC == 128)
-    tmem_ld128(ts, *reinterpret_cast<uint32_t(*)[128]>(r));
-  else
-    tmem_ld64(ts, *reinterpret_cast<uint32_t(*)[64]>(r));
+// Softmax of one tile's half (64 columns, MASK: keys at or past `valid` masked) for this
+// thread's row, in one pass: load the 64 S values, row max, lazy max update, then
+// P = 2^(S*scale*log2e - m) with packed fp32x2 FMAs, MUFU ex2 and packed sums, stored as
+// bf16 pairs over the first 32 of the columns just read.  A rescale of O_k waits for the
+// P.V of the previous tile (`pv_prev`, phase parity `pv_par`), which completes every
+// earlier product;
+// if that wait gives up, the rescale is skipped and false is returned (the kernel is
+// aborting; the caller leaves at the next group wait).
+template <int D, bool MASK>
+__device__ __forceinline__ bool softmax_tile(uint32_t ts, uint32_t to, int valid, bool fresh, float sl2, float& m,
+                                             float& l, uint64_t* pv_prev, uint32_t pv_par, volatile int* abort_flag,
+                                             int* status) {
+  uint32_t r[kHalfN];
+  tmem_ld64(ts, r);
   if (MASK) {
 #pragma unroll
-    for (int i = 0; i < NC; ++i)
+    for (int i = 0; i < kHalfN; ++i)
       if (i >= valid) r[i] = __float_as_uint(-INFINITY);
   }
   float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
 #pragma unroll
-  for (int i = 0; i < NC; i += 8) {
+  for (int i = 0; i < kHalfN; i += 8) {
     a0 = fmax3(a0, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
     a1 = fmax3(a1, __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
     a2 = fmax3(a2, __uint_as_float(r[i + 4]), __uint_as_float(r[i + 5]));
@@ -376,7 +453,7 @@ __device__ __forceinline__ void softmax_tile(uint32_t ts, uint32_t to, int valid
   const float m_tile = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3)) * sl2;
   float alpha = 1.f;
   bool rescale = false;
-  if (first) {
+  if (fresh) {
     m = m_tile;
   } else {
     const bool need = m_tile > m + kRescaleThreshold;
@@ -391,14 +468,28 @@ __device__ __forceinline__ void softmax_tile(uint32_t ts, uint32_t to, int valid
   const uint64_t negm2 = f2_pack(-m, -m);
   uint64_t sum_a = 0, sum_b = 0;  // packed fp32 pairs (+0.0f, +0.0f)
 #pragma unroll
-  for (int c = 0; c < NC / 32; ++c) {
+  for (int c = 0; c < kHalfN / 32; ++c) {
     uint32_t pk[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const int k = c * 32 + 2 * i;
       const uint64_t x = fma_f32x2(f2_pack(__uint_as_float(r[k]), __uint_as_float(r[k + 1])), scale2, negm2);
-      const float p0 = ex2_approx(f2_lo(x));
-      const float p1 = ex2_approx(f2_hi(x));
+      float p0, p1;
+      if (!MASK && kEmuEvery > 0 && (i % kEmuEvery) == kEmuEvery - 1) {
+        // x >= -125 keeps 2^n a normal number; smaller terms are below 2^-125 of a sum >= 1.
+        const uint64_t xc = f2_pack(fmaxf(f2_lo(x), -125.f), fmaxf(f2_hi(x), -125.f));
+        const uint64_t shift = f2_pack(12582912.f, 12582912.f);
+        const uint64_t t = add_f32x2(xc, shift);
+        const uint64_t fr = add_f32x2(xc, add_f32x2(shift, f2_pack(-f2_lo(t), -f2_hi(t))));
+        uint64_t q = fma_f32x2(fr, f2_pack(kExp2C3, kExp2C3), f2_pack(kExp2C2, kExp2C2));
+        q = fma_f32x2(fr, q, f2_pack(kExp2C1, kExp2C1));
+        q = fma_f32x2(fr, q, f2_pack(kExp2C0, kExp2C0));
+        p0 = __uint_as_float(__float_as_uint(f2_lo(q)) + (__float_as_uint(f2_lo(t)) << 23));
+        p1 = __uint_as_float(__float_as_uint(f2_hi(q)) + (__float_as_uint(f2_hi(t)) << 23));
+      } else {
+        p0 = ex2_approx(f2_lo(x));
+        p1 = ex2_approx(f2_hi(x));
+      }
       const uint64_t pp = f2_pack(p0, p1);
       if (i & 1)
         sum_b = add_f32x2(sum_b, pp);
@@ -411,10 +502,14 @@ __device__ __forceinline__ void softmax_tile(uint32_t ts, uint32_t to, int valid
   const uint64_t sum = add_f32x2(sum_a, sum_b);
   l += f2_lo(sum) + f2_hi(sum);
   if (rescale) {
-    // Rows whose max grew by more than 8 rescale O by alpha (1 for the other rows of the
-    // warp).  O holds every earlier P.V product (see the MMA issue order), and the P.V of
-    // this tile is issued only after P_ready, i.e. after these stores complete.
-#pragma unroll
+    // Rows whose max grew by more than 8 rescale O_k by alpha (1 for the other rows of
+    // the warp).  This tile's P.V is issued only after p_ready, i.e. after these stores.
+    if (!warp_wait(pv_prev, pv_par, abort_flag, status)) {
+      tmem_wait_st();
+      return false;
+    }
+    tc_fence_after();
+#pragma unroll 1
     for (int c = 0; c < D / 32; ++c) {
       uint32_t o[32];
       tmem_ld32(to + c * 32, o);
@@ -424,14 +519,15 @@ __device__ __forceinline__ void softmax_tile(uint32_t ts, uint32_t to, int valid
     }
   }
   tmem_wait_st();
+  return true;
 }
 
-// Write 32 columns (block cc) of this thread's output row, scaled by 1/l: fp32 or bf16,
-// with 32-byte stores when the output base is 32-byte aligned (p.out_v8), else 16-byte.
+// Write 32 columns (block cc) of this thread's output row (values already normalised):
+// fp32 or bf16, with 32-byte stores when the output base is 32-byte aligned (p.out_v8),
+// else 16-byte.
 template <int D>
-__device__ __forceinline__ void store_row(const AttnParams& p, size_t o_off, const uint32_t (&r)[32], int cc,
-                                          float inv_l) {
-  auto sc = [&](int i) { return __uint_as_float(r[i]) * inv_l; };
+__device__ __forceinline__ void store_row(const AttnParams& p, size_t o_off, const uint32_t (&r)[32], int cc) {
+  auto sc = [&](int i) { return __uint_as_float(r[i]); };
   if (p.out_f32) {
     float* o = static_cast<float*>(p.out) + o_off + cc * 32;
     if (p.out_v8) {
@@ -480,71 +576,80 @@ __device__ __forceinline__ void write_empty_row(const AttnParams& p, int c, cons
         -INFINITY;
 }
 
-// Softmax warpgroup w: every tile of every block of every unit; at a block's end it hands
-// the row's (m, l) to the epilogue warpgroup and carries on with the next block.
+// Softmax warpgroup k (key half k): every tile of every block of every unit; at a
+// segment's end it hands the row's (m_k, l_k) to the epilogue warpgroup.
 template <int D>
 __device__ __forceinline__ void attn_softmax(const AttnParams& p, uint8_t* smem, uint64_t* bars, uint32_t tmem,
                                              volatile int* abort_flag) {
   using L = AttnSmem<D>;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int w = warp >> 2;        // warpgroup = Q tile of the pair
+  const int kh = warp >> 2;       // key half
   const int quarter = warp & 3;   // TMEM lane quarter
   const int row = quarter * 32 + lane;
   const uint32_t lanes = static_cast<uint32_t>(quarter * 32) << 16;
-  const uint32_t ts = tmem + lanes + w * kBN;          // S_w
-  const uint32_t to = tmem + lanes + 256 + w * 128;    // O_w
-  float2* stat = reinterpret_cast<float2*>(smem + L::kStat) + w * 2 * kBM;
+  const uint32_t to = tmem + lanes + kTmemO + kh * 128;  // O_k
+  float2* stat = reinterpret_cast<float2*>(smem + L::kStat) + kh * 2 * kBM;
   const float sl2 = p.scale_log2;
-  uint32_t g = 0, nch = 0;
+  const int gbar = kBarSoftmax0 + kh;
+  uint32_t g = 0;     // tiles seen
+  uint32_t nch = 0;   // segments finished
+  bool alive = true;  // false once a wait of this thread gave up
 
   for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
     const UnitCoord uc = decode_unit(u, p);
-    const int s_row = (uc.qp * kQTiles + w) * kBM + row;
-    float m = -INFINITY;  // running max of S*scale*log2e (possibly stale by < 8)
+    const int s_row = uc.qt * kBM + row;
+    float m = -INFINITY;  // running max of S*scale*log2e over this half's keys (stale by < 8)
     float l = 0.f;        // running sum of 2^(S*scale*log2e - m)
-    if (p.fuse && p.first_c < 0 && s_row < p.Sq) write_empty_row<D>(p, 0, uc, s_row);  // no keys at all
+    bool fresh = true;    // no key of this half seen yet in the segment
+    if (kh == 0 && p.fuse && p.first_c < 0 && s_row < p.Sq) write_empty_row<D>(p, 0, uc, s_row);  // no keys
     for (int c = 0; c < p.n_chunks; ++c) {
       const int n_kv = block_tiles(p, c);
       if (n_kv == 0) {  // no keys: O = 0, lse = -inf (fused: the block simply adds nothing)
-        if (!p.fuse && s_row < p.Sq) write_empty_row<D>(p, c, uc, s_row);
+        if (kh == 0 && !p.fuse && s_row < p.Sq) write_empty_row<D>(p, c, uc, s_row);
         continue;
       }
       if (!p.fuse || c == p.first_c) {
         m = -INFINITY;
         l = 0.f;
+        fresh = true;
       }
       for (int j = 0; j < n_kv; ++j, ++g) {
         const Tile t = make_tile(p, c, j);
-        if (!warp_wait(bars + kSFull + w, g & 1, abort_flag, p.status)) return;
+        const int sb = g & 1;
+        if (!group_wait(bars + kQkDone + sb, (g >> 1) & 1, gbar, alive, abort_flag, p.status)) return;
         tc_fence_after();
-        if (t.valid() == 128)
-          softmax_tile<D, 128, false>(ts, to, t.valid(), t.first(), sl2, m, l);
-        else if (t.valid() > 64)
-          softmax_tile<D, 128, true>(ts, to, t.valid(), t.first(), sl2, m, l);
-        else if (t.valid() == 64)
-          softmax_tile<D, 64, false>(ts, to, t.valid(), t.first(), sl2, m, l);
-        else
-          softmax_tile<D, 64, true>(ts, to, t.valid(), t.first(), sl2, m, l);
+        const int vh = half_valid(t.valid(), kh);
+        if (vh > 0) {
+          const uint32_t ts = tmem + lanes + sb * kBN + kh * kHalfN;
+          // A rescale (never on a segment's first tile, so g >= 1) waits for PV(g-1).
+          uint64_t* pv_prev = bars + kPvDone + ((g - 1) & 1);
+          const uint32_t pv_par = ((g - 1) >> 1) & 1;
+          const bool ok = vh == kHalfN
+                              ? softmax_tile<D, false>(ts, to, vh, fresh, sl2, m, l, pv_prev, pv_par, abort_flag, p.status)
+                              : softmax_tile<D, true>(ts, to, vh, fresh, sl2, m, l, pv_prev, pv_par, abort_flag, p.status);
+          alive = alive && ok;
+          fresh = false;
+        }
         tc_fence_before();
-        mbar_arrive(bars + kPReady + w);
+        mbar_arrive(bars + kPReady + sb * 2 + kh);
       }
       if (p.fuse && c != p.last_c) continue;  // the segment goes on with the next block
-      // Hand (m, l) of this block to the epilogue warpgroup.  First wait until the epilogue
-      // has finished the previous block (it releases O_w only after reading that block's
-      // stats): without this wait, blocks of a single tile let this warpgroup run two
-      // stat_ready phases ahead of the epilogue, which a parity wait cannot tell apart.
-      if (nch > 0 && !warp_wait(bars + kOFree + w, (nch - 1) & 1, abort_flag, p.status)) return;
+      // Hand (m, l) to the epilogue.  First wait until it has finished the previous
+      // segment (it releases O only after reading that segment's stats): without this
+      // wait, one-tile segments let this warpgroup run two stat_ready phases ahead of the
+      // epilogue, which a parity wait cannot tell apart.
+      if (nch > 0 && !group_wait(bars + kOFree, (nch - 1) & 1, gbar, alive, abort_flag, p.status)) return;
       stat[(nch & 1) * kBM + row] = make_float2(m, l);
-      mbar_arrive(bars + kStatReady + w);
+      mbar_arrive(bars + kStatReady);
       ++nch;
     }
   }
 }
 
-// Epilogue warpgroup: for every non-empty block and both Q tiles, wait for the block's
-// last P.V and its (m, l), read O_w from TMEM 32 columns at a time, write O/l and the LSE,
-// then release O_w for the next block's first P.V.
+// Epilogue warpgroup: for every segment, wait for its last P.V and both halves' (m, l),
+// merge O_0 and O_1 32 columns at a time, write O and the LSE, then release O for the
+// next segment's first P.V.
 template <int D>
 __device__ __forceinline__ void attn_epilogue(const AttnParams& p, uint8_t* smem, uint64_t* bars, uint32_t tmem,
                                               volatile int* abort_flag) {
@@ -554,39 +659,56 @@ __device__ __forceinline__ void attn_epilogue(const AttnParams& p, uint8_t* smem
   const int quarter = warp & 3;
   const int row = quarter * 32 + lane;
   const uint32_t lanes = static_cast<uint32_t>(quarter * 32) << 16;
+  const uint32_t to0 = tmem + lanes + kTmemO;
+  const uint32_t to1 = to0 + 128;
   const float2* stat = reinterpret_cast<const float2*>(smem + L::kStat);
   uint32_t nch = 0;
   if (p.tiles_per_unit == 0) return;
   for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
     const UnitCoord uc = decode_unit(u, p);
+    const int s_row = uc.qt * kBM + row;
+    const bool row_ok = s_row < p.Sq;
     for (int c0 = 0; c0 < p.n_chunks; ++c0) {
       if (block_tiles(p, c0) == 0) continue;
       if (p.fuse && c0 != p.last_c) continue;  // one merged output per unit
       const int c = p.fuse ? 0 : c0;             // output block index
+      if (!group_wait(bars + kStatReady, nch & 1, kBarEpilogue, true, abort_flag, p.status, 64)) return;
+      if (!group_wait(bars + kODone, nch & 1, kBarEpilogue, true, abort_flag, p.status, 64)) return;
+      tc_fence_after();
+      const float2 s0 = stat[(nch & 1) * kBM + row];
+      const float2 s1 = stat[(2 + (nch & 1)) * kBM + row];
+      // Half 0 always holds a key of a non-empty segment (l_0 >= 1); half 1 is empty when
+      // every tile of the segment has at most 64 keys, and then O_1 was never written.
+      const bool has1 = s1.y > 0.f;  // the same for every row
+      const float mx = has1 ? fmaxf(s0.x, s1.x) : s0.x;
+      const float w0 = ex2_approx(s0.x - mx);
+      const float w1 = has1 ? ex2_approx(s1.x - mx) : 0.f;
+      const float lsum = s0.y * w0 + s1.y * w1;
+      const float inv = 1.f / lsum;
+      const float c0f = w0 * inv, c1f = w1 * inv;
+      const size_t o_off = static_cast<size_t>(c) * p.out_chunk_stride +
+                           ((static_cast<size_t>(uc.b) * p.Sq + s_row) * p.H + uc.h) * D;
 #pragma unroll 1
-      for (int w = 0; w < kQTiles; ++w) {
-        if (!warp_wait(bars + kStatReady + w, nch & 1, abort_flag, p.status)) return;
-        if (!warp_wait(bars + kODone + w, nch & 1, abort_flag, p.status)) return;
-        tc_fence_after();
-        const float2 ml = stat[(w * 2 + (nch & 1)) * kBM + row];
-        const float inv_l = 1.f / ml.y;
-        const int s_row = (uc.qp * kQTiles + w) * kBM + row;
-        const bool row_ok = s_row < p.Sq;
-        const size_t o_off = static_cast<size_t>(c) * p.out_chunk_stride +
-                             ((static_cast<size_t>(uc.b) * p.Sq + s_row) * p.H + uc.h) * D;
-        const uint32_t to = tmem + lanes + 256 + w * 128;
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(to0 + cc * 32, r);
+        if (__any_sync(0xffffffffu, has1)) {
+          uint32_t r1[32];
+          tmem_ld32(to1 + cc * 32, r1);
 #pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t r[32];
-          tmem_ld32(to + cc * 32, r);
-          if (row_ok) store_row<D>(p, o_off, r, cc, inv_l);
+          for (int i = 0; i < 32; ++i)
+            r[i] = __float_as_uint(fmaf(__uint_as_float(r[i]), c0f, has1 ? __uint_as_float(r1[i]) * c1f : 0.f));
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * c0f);
         }
-        tc_fence_before();
-        mbar_arrive(bars + kOFree + w);
-        if (row_ok && p.lse)
-          p.lse[static_cast<size_t>(c) * p.lse_chunk_stride + (static_cast<size_t>(uc.b) * p.H + uc.h) * p.Sq +
-                s_row] = (ml.x + log2f(ml.y)) * 0.69314718055994530942f;
+        if (row_ok) store_row<D>(p, o_off, r, cc);
       }
+      tc_fence_before();
+      mbar_arrive(bars + kOFree);
+      if (row_ok && p.lse)
+        p.lse[static_cast<size_t>(c) * p.lse_chunk_stride + (static_cast<size_t>(uc.b) * p.H + uc.h) * p.Sq +
+              s_row] = (mx + log2f(lsum)) * 0.69314718055994530942f;
       ++nch;
     }
   }
@@ -607,22 +729,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int warp = threadIdx.x >> 5;
 
   if (threadIdx.x == 0) {
-    mbar_init(bars + kQFull, 1);    // TMA transaction count
-    mbar_init(bars + kQEmpty, 1);   // MMA commit
     for (int s = 0; s < kStages; ++s) {
+      mbar_init(bars + kQFull + s, 1);   // TMA transaction count
+      mbar_init(bars + kQEmpty + s, 1);  // MMA commit after the unit's last QK
       mbar_init(bars + kKFull + s, 1);
-      mbar_init(bars + kKEmpty + s, 1);
       mbar_init(bars + kVFull + s, 1);
-      mbar_init(bars + kVEmpty + s, 1);
+      mbar_init(bars + kQkDone + s, 1);  // QK thread commit after S of a tile in slot s
+      mbar_init(bars + kPvDone + s, 1);  // P.V thread commit after P.V of a tile in slot s
     }
-    for (int w = 0; w < kQTiles; ++w) {
-      mbar_init(bars + kSFull + w, 1);     // MMA commit after QK_w
-      mbar_init(bars + kPReady + w, 128);  // the 128 threads of softmax warpgroup w
-      mbar_init(bars + kODone + w, 1);     // MMA commit after a block's last PV_w
-      mbar_init(bars + kOFree + w, 128);   // the epilogue warpgroup has read O_w
-      mbar_init(bars + kStatReady + w, 128);  // warpgroup w has written a block's (m, l)
-    }
+    for (int i = 0; i < 4; ++i) mbar_init(bars + kPReady + i, 128);  // softmax warpgroup stored P
+    mbar_init(bars + kODone, 1);       // MMA commit after a segment's last P.V
+    mbar_init(bars + kOFree, 128);     // the epilogue warpgroup has read O
+    mbar_init(bars + kStatReady, 256); // both softmax warpgroups wrote a segment's (m, l)
     mbar_init(bars + kDrain, 1);
+    mbar_init(bars + kDrainPV, 1);
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -630,8 +750,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (warp == kProducerWarp && (threadIdx.x & 31) == 0) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
-    tma_prefetch_desc(&tm_v);
   }
+  if (warp == kVProducerWarp && (threadIdx.x & 31) == 0) tma_prefetch_desc(&tm_v);
   if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
@@ -643,16 +763,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   // Producer and MMA roles run on lane 0 of their warp; the other lanes wait at the
   // __syncwarp so that each warp is converged again for the teardown below.
-  // Warps 10 and 11 only give their registers back to the softmax warpgroups.
   if (warp >= kEpilogueWarp0) {
     regs_decrease<kEpilogueRegs>();
     attn_epilogue<D>(p, smem, bars, tmem, abort_flag);
-  } else if (warp >= kQTiles * 4) {
+  } else if (warp >= 8) {
     regs_decrease<kControlRegs>();
     if (warp == kProducerWarp) {
-      if ((threadIdx.x & 31) == 0) attn_producer<D>(&tm_q, &tm_k, &tm_v, p, smem, bars, abort_flag);
+      if ((threadIdx.x & 31) == 0) attn_producer_qk<D>(&tm_q, &tm_k, p, smem, bars, abort_flag);
+    } else if (warp == kVProducerWarp) {
+      if ((threadIdx.x & 31) == 0) attn_producer_v<D>(&tm_v, p, smem, bars, abort_flag);
     } else if (warp == kMmaWarp) {
-      if ((threadIdx.x & 31) == 0) attn_mma<D>(p, smem, bars, tmem, abort_flag);
+      if ((threadIdx.x & 31) == 0) attn_mma_qk<D>(p, smem, bars, tmem, abort_flag);
+    } else if (warp == kPvWarp) {
+      if ((threadIdx.x & 31) == 0) attn_mma_pv<D>(p, smem, bars, tmem, abort_flag);
     }
     __syncwarp();
   } else {

@@ -114,8 +114,8 @@ cp_status launch_attn(const void* q, const void* k, const void* v, const int* bo
   p.H = H;
   p.Sq = Sq;
   p.n_chunks = n_chunks;
-  p.n_qp = (Sq + kQTiles * kBM - 1) / (kQTiles * kBM);
-  p.n_units = B * H * p.n_qp;
+  p.n_qt = (Sq + kBM - 1) / kBM;
+  p.n_units = B * H * p.n_qt;
   p.tiles_per_unit = 0;
   for (int i = 0; i < n_chunks; ++i) p.tiles_per_unit += (bounds[i + 1] - bounds[i] + kBN - 1) / kBN;
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
