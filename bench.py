@@ -35,6 +35,27 @@ WORKLOAD = "flux_1024_ring8_ulysses8"
 METRIC = "attention TFLOP/s (4*B*H*Sq*Skv*D) and % of B200 BF16 peak; merge/permute GB/s"
 UNIT = "TFLOP/s"
 
+# DRAM traffic of the timed attention launch (8 ring blocks, FLUX B1), from one ncu capture
+# of the same kernel on the B2 shape (profiles/attn_fwd_sm100__flux_b2_ring8.md):
+# dram__bytes_read.sum + dram__bytes_write.sum = 185.78 + 861.37 MB, halved to one B1 launch
+# (the B1 launch processes half the units; Q/K/V reads and partial writes scale with them).
+# It describes only the kernel source it was captured on, identified by its SHA-256.
+ATTN_TRAFFIC = {
+    "kernel_sha256": "8f5d0b897bd65637f466a9f0c3b0ae5212c8f95804f07fa503d6956c61afcf98",
+    "bytes_per_launch": (185_780_224 + 861_372_160) // 2,
+}
+
+
+def attn_traffic():
+    """Measured DRAM bytes per attention launch, or None if the kernel changed since."""
+    import hashlib
+
+    src = os.path.join(os.path.dirname(os.path.abspath(__file__)), "context_attention_dit_b200", "csrc",
+                       "attn_fwd_sm100.cuh")
+    with open(src, "rb") as f:
+        digest = hashlib.sha256(f.read()).hexdigest()
+    return ATTN_TRAFFIC["bytes_per_launch"] if digest == ATTN_TRAFFIC["kernel_sha256"] else None
+
 
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -323,7 +344,8 @@ def run_ours(args):
                 "frac_of_spec_2250": round(attn_tflops / 2250.0, 4),
                 "peak_source": peaks["source"] + " (burst bf16 GEMM)",
                 "flop_per_launch": flop,
-                "traffic": None,
+                "traffic": attn_traffic(),
+                "traffic_unit": "bytes per launch (ncu dram read + write)",
             },
             "kernels": {
                 "attn_ring1_tflops": round(ring1_tflops, 2),

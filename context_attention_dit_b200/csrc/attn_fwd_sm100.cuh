@@ -72,7 +72,8 @@ constexpr int kMaxChunks = 64;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // 2^x on the FMA pipe for one pair in kEmuEvery of a tile without masked keys (0: off):
 // n = rint(x) by the 1.5*2^23 shift, f = x - n in [-1/2, 1/2], 2^f by a degree-3 minimax
-// polynomial (relative error 7.5e-5, fitted for this kernel), 2^n added to the exponent.
+// polynomial (relative error 7.5e-5; context_attention_dit_b200/exp2_poly_fit.py prints the
+// coefficients), 2^n added to the exponent.
 constexpr int kEmuEvery = 4;
 constexpr float kExp2C0 = 0.9999280571937561f;
 constexpr float kExp2C1 = 0.6932608485221863f;
@@ -108,7 +109,7 @@ struct AttnSmem {
   static constexpr int kV = kK + kStages * kTileBytes;   // kStages V stages
   static constexpr int kStat = kV + kStages * kTileBytes;  // float2 [2 halves][2 parities][kBM]: (m, l)
   static constexpr int kBar = kStat + 2 * 2 * kBM * 8;
-  static constexpr int kNumBars = 21;
+  static constexpr int kNumBars = 19;
   static constexpr int kUsed = kBar + kNumBars * 8 + 16;
   // Request enough that at most one CTA fits per SM (the kernel allocates all 512 TMEM
   // columns), plus 1 KB for aligning the base to the 128B-swizzle atom.
@@ -121,10 +122,11 @@ struct AttnSmem {
 //                 producer);
 //   pv_done[t%2]  after O += P(t) V(t): V stage t%2 is free (V producer), S buffer t%2 is
 //                 free for QK(t+2), O holds every product up to tile t (softmax rescale).
-// p_ready is [S buffer][half].
+// p_ready is per S buffer.  Warp-level signals (p_ready, stat_ready, o_free) are arrived
+// by one lane per warp after __syncwarp, so a barrier sees one arrival per warp.
 enum : int {
   kQFull = 0, kQEmpty = 2, kKFull = 4, kVFull = 6, kQkDone = 8, kPvDone = 10, kPReady = 12,
-  kODone = 16, kOFree = 17, kStatReady = 18, kDrain = 19, kDrainPV = 20
+  kODone = 14, kOFree = 15, kStatReady = 16, kDrain = 17, kDrainPV = 18
 };
 
 struct UnitCoord {
@@ -212,6 +214,13 @@ __device__ __forceinline__ bool group_wait(uint64_t* bar, uint32_t parity, int i
   bool ok = alive;
   if ((threadIdx.x & 127) < 32 && ok) ok = mbar_wait(bar, parity, abort_flag, status, sleep_ns);
   return bar_and(id, 128, ok);
+}
+
+// One arrival for the whole warp, after every lane's earlier work (ordered by the caller's
+// fences) is complete: __syncwarp orders the lanes, then lane 0 arrives.
+__device__ __forceinline__ void warp_arrive(uint64_t* bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
 
 // Wait bounded by time only (used to drain in-flight work after an abort).
@@ -337,8 +346,9 @@ __device__ __forceinline__ void attn_mma_qk(const AttnParams& p, uint8_t* smem, 
       const bool more = next_tile(p, t, nxt);
       const int kst = kc % kStages;
       const int sb = g & 1;
-      if (g >= 2 && !mbar_wait(bars + kPvDone + sb, ((g >> 1) - 1) & 1, abort_flag, p.status)) goto done;
+      // K(t) lands long before buffer t%2 frees: test it first, off the critical path.
       if (!mbar_wait(bars + kKFull + kst, (kc / kStages) & 1, abort_flag, p.status)) goto done;
+      if (g >= 2 && !mbar_wait(bars + kPvDone + sb, ((g >> 1) - 1) & 1, abort_flag, p.status)) goto done;
       tc_fence_after();
       const uint32_t d_tmem = tmem + sb * kBN;
       const uint64_t kd = sdesc_sw128(sK + kst * L::kTileBytes, 16, 1024);
@@ -385,8 +395,7 @@ __device__ __forceinline__ void attn_mma_pv(const AttnParams& p, uint8_t* smem, 
       const uint32_t ppar = (gp >> 1) & 1;
       if (t.first()) init0 = init1 = false;
       if (!mbar_wait(bars + kVFull + vst, (vc / kStages) & 1, abort_flag, p.status)) goto done;
-      if (!mbar_wait(bars + kPReady + sb * 2, ppar, abort_flag, p.status)) goto done;
-      if (!mbar_wait(bars + kPReady + sb * 2 + 1, ppar, abort_flag, p.status)) goto done;
+      if (!mbar_wait(bars + kPReady + sb, ppar, abort_flag, p.status)) goto done;
       if (t.first() && nch > 0 && !mbar_wait(bars + kOFree, (nch - 1) & 1, abort_flag, p.status)) goto done;
       tc_fence_after();
       const uint64_t vd = sdesc_sw128(sV + vst * L::kTileBytes, L::kHalfBytes, 1024);
@@ -632,7 +641,7 @@ __device__ __forceinline__ void attn_softmax(const AttnParams& p, uint8_t* smem,
           fresh = false;
         }
         tc_fence_before();
-        mbar_arrive(bars + kPReady + sb * 2 + kh);
+        warp_arrive(bars + kPReady + sb);
       }
       if (p.fuse && c != p.last_c) continue;  // the segment goes on with the next block
       // Hand (m, l) to the epilogue.  First wait until it has finished the previous
@@ -641,7 +650,7 @@ __device__ __forceinline__ void attn_softmax(const AttnParams& p, uint8_t* smem,
       // epilogue, which a parity wait cannot tell apart.
       if (nch > 0 && !group_wait(bars + kOFree, (nch - 1) & 1, gbar, alive, abort_flag, p.status)) return;
       stat[(nch & 1) * kBM + row] = make_float2(m, l);
-      mbar_arrive(bars + kStatReady);
+      warp_arrive(bars + kStatReady);
       ++nch;
     }
   }
@@ -705,7 +714,7 @@ __device__ __forceinline__ void attn_epilogue(const AttnParams& p, uint8_t* smem
         if (row_ok) store_row<D>(p, o_off, r, cc);
       }
       tc_fence_before();
-      mbar_arrive(bars + kOFree);
+      warp_arrive(bars + kOFree);
       if (row_ok && p.lse)
         p.lse[static_cast<size_t>(c) * p.lse_chunk_stride + (static_cast<size_t>(uc.b) * p.H + uc.h) * p.Sq +
               s_row] = (mx + log2f(lsum)) * 0.69314718055994530942f;
@@ -737,10 +746,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(bars + kQkDone + s, 1);  // QK thread commit after S of a tile in slot s
       mbar_init(bars + kPvDone + s, 1);  // P.V thread commit after P.V of a tile in slot s
     }
-    for (int i = 0; i < 4; ++i) mbar_init(bars + kPReady + i, 128);  // softmax warpgroup stored P
+    mbar_init(bars + kPReady + 0, 8);  // each of the 8 softmax warps stored its P
+    mbar_init(bars + kPReady + 1, 8);
     mbar_init(bars + kODone, 1);       // MMA commit after a segment's last P.V
-    mbar_init(bars + kOFree, 128);     // the epilogue warpgroup has read O
-    mbar_init(bars + kStatReady, 256); // both softmax warpgroups wrote a segment's (m, l)
+    mbar_init(bars + kOFree, 4);       // each epilogue warp has read its O rows
+    mbar_init(bars + kStatReady, 8);   // each softmax warp wrote a segment's (m, l)
     mbar_init(bars + kDrain, 1);
     mbar_init(bars + kDrainPV, 1);
     *abort_flag = 0;
