@@ -276,6 +276,41 @@ def run_ours(args):
     torch.cuda.synchronize()
     fused_ms = statistics.mean(a.elapsed_time(b) for a, b in rf[max(args.warmup, 3):])
 
+    def timed_ms(fn, reps=20):
+        evs = []
+        for i in range(max(args.warmup, 3) + reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            evs.append((a, b))
+        torch.cuda.synchronize()
+        return statistics.mean(a.elapsed_time(b) for a, b in evs[max(args.warmup, 3):])
+
+    # Unified SP: Ulysses 2 x ring 4 and Ulysses 4 x ring 2 on the same tensors, through
+    # cp_usp_sim (exchange, ring attention + merge, inverse exchange, LSE regroup).
+    usp = {}
+    for U, R in ((2, 4), (4, 2)):
+        sh = [t.reshape(B, U, S // U, H, D).permute(1, 0, 2, 3, 4).contiguous().to(dev) for t in (q_h, k_h, v_h)]
+        ws = torch.empty(binding.usp_workspace_size(U, R, B, S, H, D), dtype=torch.uint8, device=dev)
+        uo = torch.empty_like(sh[0])
+        ul = torch.empty((B, H, S), dtype=torch.float32, device=dev)
+        ub = even_bounds(S, R)
+        ms = timed_ms(lambda: binding.usp_sim(*sh, U, ub, scale=scale, workspace=ws, out=uo, out_lse=ul))
+        usp[f"usp_u{U}_r{R}_ms"] = round(ms, 4)
+        usp[f"usp_u{U}_r{R}_tflops"] = round(flop / (ms * 1e-3) / 1e12, 2)
+        del sh, ws, uo, ul
+
+    # Ulysses Anything exchange: FLUX at 1008x1008 (4481 tokens) over 4 ranks, one tensor.
+    Sa = 4481
+    xa = torch.randn(B * Sa * H * D, generator=torch.Generator().manual_seed(5)).bfloat16().to(dev)
+    ya = torch.empty_like(xa)
+    sba, hba = binding.ring_bounds(Sa, 4, anything=True), binding.ring_bounds(H, 4, anything=True)
+    any_ms = timed_ms(lambda: binding.ulysses_anything_permute(xa, 4, sba, hba, B, Sa, H, D, 0, dst=ya))
+    any_bytes = 2 * xa.numel() * xa.element_size()
+    del xa, ya
+
     # End to end through the public API with host buffers (pinned), per step:
     # H2D of the sequence-sharded Q/K/V, the hot path, D2H of O.
     hq, hk, hv = (seq_shards(t).pin_memory() for t in (q_h, k_h, v_h))
@@ -361,6 +396,9 @@ def run_ours(args):
                 "permute_inv_ms": round(statistics.mean(inv_ms), 4),
                 "permute_inv_gbs": round(inv_bytes / (statistics.mean(inv_ms) * 1e-3) / 1e9, 1),
                 "hbm_peak_gbs": peaks["hbm_gbs"],
+                **usp,
+                "anything_permute_flux1008_p4_ms": round(any_ms, 4),
+                "anything_permute_flux1008_p4_gbs": round(any_bytes / (any_ms * 1e-3) / 1e9, 1),
             },
             "e2e": {"value": round(world * flop / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},

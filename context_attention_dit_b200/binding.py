@@ -34,7 +34,8 @@ CP_MAX_CHUNKS = 64
 EXPORTS = (
     "cp_attn_fwd", "cp_attn_fwd_blocks", "cp_attn_merge", "cp_ring_sim_workspace_size", "cp_ring_sim",
     "cp_ring_sim_fused", "cp_ring_sim_static", "cp_ulysses_permute", "cp_ulysses_permute_n", "cp_ring_bounds",
-    "cp_debug_set_fault", "cp_last_device_status", "cp_status_string", "cp_version",
+    "cp_debug_set_fault", "cp_last_device_status", "cp_status_string", "cp_version", "cp_usp_sim_workspace_size",
+    "cp_usp_sim", "cp_ulysses_anything_permute",
 )
 
 _lib = None
@@ -63,9 +64,13 @@ def load() -> ctypes.CDLL:
     lib.cp_ring_sim_workspace_size.restype = sz
     lib.cp_ring_sim.argtypes = [vp, vp, vp, ip, i, vp, vp, i, i, i, i, i, f, i, vp, sz, vp]
     lib.cp_ring_sim_fused.argtypes = [vp, vp, vp, ip, i, vp, vp, i, i, i, i, i, f, i, vp]
+    lib.cp_usp_sim_workspace_size.argtypes = [i, i, i, i, i, i, i]
+    lib.cp_usp_sim_workspace_size.restype = sz
+    lib.cp_usp_sim.argtypes = [vp, vp, vp, i, ip, i, vp, vp, i, i, i, i, f, i, vp, sz, vp]
     lib.cp_ring_sim_fused.restype = ctypes.c_int
     lib.cp_ring_sim_static.argtypes = [vp, vp, vp, ip, i, vp, vp, i, i, i, i, i, f, i, vp]
     lib.cp_ulysses_permute.argtypes = [vp, vp, i, i, i, i, i, i, i, vp]
+    lib.cp_ulysses_anything_permute.argtypes = [vp, vp, i, ip, ip, i, i, i, i, i, i, vp]
     lib.cp_ulysses_permute_n.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), i, i, i, i, i, i, i, i, vp]
     lib.cp_ulysses_permute_n.restype = ctypes.c_int
     lib.cp_ring_bounds.argtypes = [i, i, i, ip]
@@ -213,6 +218,47 @@ def ring_sim(q, k, v, chunk_bounds: Sequence[int], scale: Optional[float] = None
     return out, out_lse, workspace
 
 
+def usp_workspace_size(degree: int, n_chunks: int, B: int, S: int, H: int, D: int, out_dtype=torch.bfloat16) -> int:
+    return int(load().cp_usp_sim_workspace_size(degree, n_chunks, B, S, H, D, _out_code(out_dtype)))
+
+
+def usp_sim(q, k, v, degree: int, chunk_bounds: Sequence[int], scale: Optional[float] = None,
+            out_dtype=torch.bfloat16, workspace=None, out=None, out_lse=None):
+    """Ulysses (``degree``) x ring (``chunk_bounds`` over the whole sequence) attention.
+
+    q, k, v: sequence-sharded ``[degree, B, S/degree, H, D]`` bf16 (shard p = tokens
+    ``[p*S/degree, (p+1)*S/degree)``).  Returns ``(out, lse, workspace)``: out in the same
+    layout, lse ``[B, H, S]`` fp32.
+    """
+    for name, t in (("query", q), ("key", k), ("value", v)):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.bfloat16 or t.dim() != 5:
+            raise ValueError(f"{name} must be a 5-D bf16 CUDA tensor [degree, B, S/degree, H, D]")
+        if not t.is_contiguous() or t.shape != q.shape or t.device != q.device:
+            raise ValueError("query, key and value must be contiguous, of one shape, on one device")
+    P, B, Sp, H, D = q.shape
+    if P != degree:
+        raise ValueError(f"leading dimension {P} != degree {degree}")
+    S = P * Sp
+    code = _out_code(out_dtype)
+    scale = float(D ** -0.5 if scale is None else scale)
+    n = len(chunk_bounds) - 1
+    if n < 1:
+        raise ValueError("chunk_bounds needs at least two entries")
+    bounds = (ctypes.c_int * (n + 1))(*[int(c) for c in chunk_bounds])
+    need = usp_workspace_size(degree, n, B, S, H, D, out_dtype)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+    if out_lse is None:
+        out_lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    st = load().cp_usp_sim(_ptr(q), _ptr(k), _ptr(v), degree, bounds, n, _ptr(out), _ptr(out_lse), B, S, H, D, scale,
+                           code, _ptr(workspace), ws_bytes, ctypes.c_void_p(_stream(q)))
+    _check(st, "cp_usp_sim")
+    return out, out_lse, workspace
+
+
 def ring_sim_fused(q, k, v, chunk_bounds: Sequence[int], scale: Optional[float] = None, out_dtype=torch.bfloat16,
                    out=None, out_lse=None):
     """Ring attention over K/V blocks with the LSE merge fused into the kernel; returns ``(out, lse)``."""
@@ -345,6 +391,26 @@ def ulysses_permute_n(srcs, degree: int, direction: int, dsts=None):
                                      ctypes.c_void_p(_stream(ref)))
     _check(st, "cp_ulysses_permute_n")
     return dsts
+
+
+def ulysses_anything_permute(src, degree: int, seq_bounds: Sequence[int], head_bounds: Sequence[int], B: int, S: int,
+                             H: int, D: int, direction: int, dst=None):
+    """Ulysses exchange with unequal shards (see cp_ulysses_anything_permute): src and the
+    returned dst are packed buffers of B*S*H*D elements (1-D views)."""
+    if not isinstance(src, torch.Tensor) or not src.is_cuda or not src.is_contiguous():
+        raise ValueError("src must be a contiguous CUDA tensor")
+    if src.numel() != B * S * H * D:
+        raise ValueError(f"src has {src.numel()} elements, expected B*S*H*D = {B * S * H * D}")
+    if len(seq_bounds) != degree + 1 or len(head_bounds) != degree + 1:
+        raise ValueError("seq_bounds and head_bounds need degree + 1 entries")
+    sb = (ctypes.c_int * (degree + 1))(*[int(x) for x in seq_bounds])
+    hb = (ctypes.c_int * (degree + 1))(*[int(x) for x in head_bounds])
+    if dst is None:
+        dst = torch.empty(src.numel(), dtype=src.dtype, device=src.device)
+    st = load().cp_ulysses_anything_permute(_ptr(src), _ptr(dst), degree, sb, hb, B, S, H, D, direction,
+                                            src.element_size(), ctypes.c_void_p(_stream(src)))
+    _check(st, "cp_ulysses_anything_permute")
+    return dst.view(-1)
 
 
 def ring_bounds(S: int, n: int, anything: bool = False):

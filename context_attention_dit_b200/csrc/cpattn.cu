@@ -345,6 +345,61 @@ cp_status cp_ring_sim_static(const void* q, const void* k, const void* v, const 
                      need, stream);
 }
 
+size_t cp_usp_sim_workspace_size(int degree, int n_chunks, int B, int S, int H, int D, cp_dtype out_dtype) {
+  if (degree < 1 || n_chunks < 1 || B <= 0 || S <= 0 || H <= 0 || D <= 0 || H % degree != 0) return 0;
+  const size_t elems = static_cast<size_t>(B) * S * H * D;
+  const size_t out_bytes = out_dtype == CP_F32 ? 4 : 2;
+  return 3 * round256(elems * 2) + round256(elems * out_bytes) +
+         round256(static_cast<size_t>(B) * H * S * sizeof(float)) +
+         cp_ring_sim_workspace_size(n_chunks, degree * B, H / degree, S, D);
+}
+
+cp_status cp_usp_sim(const void* q, const void* k, const void* v, int degree, const int* chunk_bounds, int n_chunks,
+                     void* out, float* out_lse, int B, int S, int H, int D, float scale, cp_dtype out_dtype,
+                     void* workspace, size_t ws_bytes, void* stream) {
+  if (degree < 1 || B <= 0 || S <= 0 || H <= 0) return CP_ERR_INVALID_ARG;
+  if (S % degree != 0 || H % degree != 0) return CP_ERR_NOT_DIVISIBLE;
+  cp_status st = check_bounds(chunk_bounds, n_chunks, S);
+  if (st != CP_OK) return st;
+  st = check_attn_args(q, k, v, out, out_lse, B, H, S, S, D, scale, out_dtype);
+  if (st != CP_OK) return st;
+  const size_t need = cp_usp_sim_workspace_size(degree, n_chunks, B, S, H, D, out_dtype);
+  if (!workspace || ws_bytes < need) return CP_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return CP_ERR_MISALIGNED;
+  const size_t elems = static_cast<size_t>(B) * S * H * D;
+  const int out_bytes = out_dtype == CP_F32 ? 4 : 2;
+  char* w = static_cast<char*>(workspace);
+  void* qh = w;
+  void* kh = w + round256(elems * 2);
+  void* vh = w + 2 * round256(elems * 2);
+  void* oh = w + 3 * round256(elems * 2);
+  float* lse_h = reinterpret_cast<float*>(w + 3 * round256(elems * 2) + round256(elems * out_bytes));
+  char* ring_ws = reinterpret_cast<char*>(lse_h) + round256(static_cast<size_t>(B) * H * S * sizeof(float));
+  const size_t ring_bytes = ws_bytes - static_cast<size_t>(ring_ws - w);
+  // 1. First all-to-all: sequence-sharded Q, K, V -> head-sharded [P][B][S][H/P][D].
+  const void* srcs[3] = {q, k, v};
+  void* const dsts[3] = {qh, kh, vh};
+  st = cp_ulysses_permute_n(srcs, dsts, 3, degree, B, S, H, D, 0, 2, stream);
+  if (st != CP_OK) return st;
+  // 2. Ring attention over the K/V blocks, every head shard at once (batch P*B, H/P heads).
+  st = cp_ring_sim(qh, kh, vh, chunk_bounds, n_chunks, oh, out_lse ? lse_h : nullptr, degree * B, H / degree, S, S,
+                   D, scale, out_dtype, ring_ws, ring_bytes, stream);
+  if (st != CP_OK) return st;
+  // 3. Second all-to-all: head-sharded O -> sequence-sharded, as the inputs.
+  st = cp_ulysses_permute(oh, out, degree, B, S, H, D, 1, out_bytes, stream);
+  if (st != CP_OK) return st;
+  // 4. LSE [P][B][H/P][S] -> [B][H][S].
+  if (out_lse) {
+    const long long block = static_cast<long long>(H / degree) * S;
+    const long long gx = (block + 255) / 256 < 1024 ? (block + 255) / 256 : 1024;
+    if (static_cast<long long>(degree) * B > 65535) return CP_ERR_UNSUPPORTED;
+    lse_regroup_kernel<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(degree * B)), 256, 0,
+                         static_cast<cudaStream_t>(stream)>>>(lse_h, out_lse, degree, B, block);
+    if (cudaGetLastError() != cudaSuccess) return CP_ERR_CUDA;
+  }
+  return CP_OK;
+}
+
 cp_status cp_ring_sim_fused(const void* q, const void* k, const void* v, const int* chunk_bounds, int n_chunks,
                             void* out, float* out_lse, int B, int H, int Sq, int Skv, int D, float scale,
                             cp_dtype out_dtype, void* stream) {
@@ -405,6 +460,60 @@ cp_status cp_ulysses_permute_n(const void* const* srcs, void* const* dsts, int n
   else if (piece_bytes % 8 == 0)
     launch(uint2{});
   else if (piece_bytes % 4 == 0)
+    launch(uint32_t{});
+  else
+    launch(uint16_t{});
+  return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+}
+
+cp_status cp_ulysses_anything_permute(const void* src, void* dst, int degree, const int* seq_bounds,
+                                      const int* head_bounds, int B, int S, int H, int D, int direction, int elem_bytes,
+                                      void* stream) {
+  if (degree < 1 || B < 0 || S < 0 || H < 0 || D < 0 || !seq_bounds || !head_bounds) return CP_ERR_INVALID_ARG;
+  if (degree > kPermuteMaxDegree) return CP_ERR_UNSUPPORTED;
+  if (direction != 0 && direction != 1) return CP_ERR_INVALID_ARG;
+  if (elem_bytes != 2 && elem_bytes != 4) return CP_ERR_UNSUPPORTED;
+  if (seq_bounds[0] != 0 || seq_bounds[degree] != S || head_bounds[0] != 0 || head_bounds[degree] != H)
+    return CP_ERR_INVALID_ARG;
+  for (int i = 0; i < degree; ++i)
+    if (seq_bounds[i] > seq_bounds[i + 1] || head_bounds[i] > head_bounds[i + 1]) return CP_ERR_INVALID_ARG;
+  if (B == 0 || S == 0 || H == 0 || D == 0) return CP_OK;
+  if (!src || !dst) return CP_ERR_INVALID_ARG;
+  if (!aligned16(src) || !aligned16(dst)) return CP_ERR_MISALIGNED;
+  const long long total = static_cast<long long>(B) * S * H * D * elem_bytes;
+  const char* s0 = static_cast<const char*>(src);
+  const char* d0 = static_cast<const char*>(dst);
+  if (s0 < d0 + total && d0 < s0 + total) return CP_ERR_INVALID_ARG;
+  if (static_cast<long long>(degree) * B > 65535 || static_cast<long long>(H) * D >= (1LL << 31))
+    return CP_ERR_UNSUPPORTED;
+  DeviceInfo* dev = nullptr;
+  cp_status st = device_info(&dev);
+  if (st != CP_OK) return st;
+  AnyBounds bd;
+  std::memset(&bd, 0, sizeof(bd));
+  int max_sp = 0;
+  for (int i = 0; i <= degree; ++i) {
+    bd.seq[i] = seq_bounds[i];
+    bd.head[i] = head_bounds[i];
+    if (i < degree && seq_bounds[i + 1] - seq_bounds[i] > max_sp) max_sp = seq_bounds[i + 1] - seq_bounds[i];
+  }
+  const int groups = (max_sp + kPermuteRows - 1) / kPermuteRows;
+  const unsigned gy = static_cast<unsigned>(groups < 65535 ? groups : 65535);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const long long row_bytes = static_cast<long long>(D) * elem_bytes;  // a vector never crosses a head
+  auto launch = [&](auto tag) {
+    using V = decltype(tag);
+    const int ve = static_cast<int>(sizeof(V)) / elem_bytes;
+    const int row_vecs = H * D / ve;
+    const dim3 grid((row_vecs + kPermuteThreads - 1) / kPermuteThreads, gy, degree * B);
+    ulysses_anything_kernel<V><<<grid, kPermuteThreads, 0, cs>>>(static_cast<const V*>(src), static_cast<V*>(dst), bd,
+                                                                 degree, B, S, H, D, ve, direction);
+  };
+  if (row_bytes % 16 == 0)
+    launch(uint4{});
+  else if (row_bytes % 8 == 0)
+    launch(uint2{});
+  else if (row_bytes % 4 == 0 && elem_bytes <= 4)
     launch(uint32_t{});
   else
     launch(uint16_t{});

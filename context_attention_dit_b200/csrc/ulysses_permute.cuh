@@ -69,4 +69,76 @@ __global__ void __launch_bounds__(kPermuteThreads)
   }
 }
 
+// The exchange for shards of unequal size ("Ulysses Anything Attention": the sequence
+// length and head count need not be divisible by the degree).  Sequence shard p holds
+// tokens [seq[p], seq[p+1]) of every head, packed at element offset B*seq[p]*H*D as
+// [B][S_p][H][D]; head shard q holds heads [head[q], head[q+1]) of every token, packed at
+// B*S*head[q]*D as [B][S][H_q][D].  With equal shards both are the stacked layouts above.
+constexpr int kPermuteMaxDegree = 64;
+
+struct AnyBounds {
+  int seq[kPermuteMaxDegree + 1];
+  int head[kPermuteMaxDegree + 1];
+};
+
+// Walks the sequence-sharded rows: grid.x covers the vectors of a token row (VE elements
+// each, D a multiple of VE so no vector crosses a head), grid.y groups of kPermuteRows rows
+// of a shard (strided by gridDim.y), grid.z = p * B + b.  Each thread finds the head group
+// of its vector once and reuses it for every row.
+template <typename V>
+__global__ void __launch_bounds__(kPermuteThreads)
+    ulysses_anything_kernel(const V* __restrict__ src, V* __restrict__ dst, const __grid_constant__ AnyBounds bd,
+                            int P, int B, int S, int H, int D, int VE, int direction) {
+  const int row_vecs = H * D / VE;
+  const int i = blockIdx.x * kPermuteThreads + threadIdx.x;
+  if (i >= row_vecs) return;
+  const int p = blockIdx.z / B;
+  const int b = blockIdx.z - p * B;
+  const int s0 = bd.seq[p];
+  const int Sp = bd.seq[p + 1] - s0;
+  const long long e = static_cast<long long>(i) * VE;  // element within the token row
+  const int h = static_cast<int>(e / D);
+  int q = 0;
+  while (bd.head[q + 1] <= h) ++q;  // the group holding head h (groups may be empty)
+  const int hq = bd.head[q];
+  const long long Hq = bd.head[q + 1] - hq;
+  const long long w = e - static_cast<long long>(hq) * D;  // element within the group's row
+  // Vector offsets of row s_local of this (p, b) on each side.
+  const long long x0 = (static_cast<long long>(B) * s0 * H * D + static_cast<long long>(b) * Sp * H * D + e) / VE;
+  const long long xs = static_cast<long long>(H) * D / VE;
+  const long long y0 = (static_cast<long long>(B) * S * hq * D + (static_cast<long long>(b) * S + s0) * Hq * D + w) / VE;
+  const long long ys = Hq * D / VE;
+  for (int sl0 = blockIdx.y * kPermuteRows; sl0 < Sp; sl0 += gridDim.y * kPermuteRows) {
+    V v[kPermuteRows];
+#pragma unroll
+    for (int r = 0; r < kPermuteRows; ++r) {
+      const int sl = sl0 + r;
+      if (sl < Sp) v[r] = direction == 0 ? src[x0 + sl * xs] : src[y0 + sl * ys];
+    }
+#pragma unroll
+    for (int r = 0; r < kPermuteRows; ++r) {
+      const int sl = sl0 + r;
+      if (sl < Sp) {
+        if (direction == 0)
+          dst[y0 + sl * ys] = v[r];
+        else
+          dst[x0 + sl * xs] = v[r];
+      }
+    }
+  }
+}
+
+// LSE of attention computed on the head-sharded layout, [P][B][H/P][S] (head group p =
+// heads [p*H/P, (p+1)*H/P)), regrouped to [B][H][S]: the (p, b) block of (H/P)*S floats is
+// contiguous on both sides.  grid.y = p*B + b; grid.x strides over the block.
+__global__ void __launch_bounds__(256) lse_regroup_kernel(const float* __restrict__ src, float* __restrict__ dst,
+                                                          int P, int B, long long block) {
+  const int pb = blockIdx.y;
+  const int p = pb / B;
+  const int b = pb - p * B;
+  const float* s = src + static_cast<long long>(pb) * block;
+  float* d = dst + (static_cast<long long>(b) * P + p) * block;
+  for (long long i = blockIdx.x * 256LL + threadIdx.x; i < block; i += gridDim.x * 256LL) d[i] = s[i];
+}
+
 }  // namespace cpattn

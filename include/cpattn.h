@@ -155,6 +155,33 @@ CP_API cp_status cp_ring_sim_fused(const void* q, const void* k, const void* v, 
                             int n_chunks, void* out, float* out_lse, int B, int H, int Sq, int Skv,
                             int D, float scale, cp_dtype out_dtype, void* stream);
 
+/* Size in bytes of the workspace cp_usp_sim needs (0 for invalid sizes or H % degree != 0). */
+CP_API size_t cp_usp_sim_workspace_size(int degree, int n_chunks, int B, int S, int H, int D,
+                                        cp_dtype out_dtype);
+
+/*
+ * cp_usp_sim - unified sequence parallelism (Ulysses x ring) simulated on one GPU.
+ *
+ * Source: "Context parallelism", section "Unified Attention": an all-to-all regroups heads
+ * and tokens, Ring Attention runs on the result, and the reverse all-to-all restores the
+ * layout; the GPUs form a ulysses_degree x ring_degree grid.  Here: the Ulysses exchange of
+ * cp_ulysses_permute (degree `degree`) on Q, K, V; cp_ring_sim over the K/V blocks
+ * `chunk_bounds` on every head shard at once; the inverse exchange of O; the LSE regrouped
+ * to the unsharded layout.  The result equals unsplit attention up to fp32 rounding order.
+ * q, k, v:     bf16, sequence-sharded and stacked rank-major, [degree][B][S/degree][H][D]
+ *              (shard p = tokens [p*S/degree, (p+1)*S/degree)), 16-byte aligned.
+ * chunk_bounds: HOST int[n_chunks+1], the ring blocks over the whole sequence [0, S]
+ *              (as cp_ring_sim, Skv = S).
+ * out:         same layout as q, out_dtype (CP_BF16 or CP_F32).
+ * out_lse:     fp32 [B][H][S] (natural log), or NULL.
+ * workspace:   cp_usp_sim_workspace_size(...) bytes, 16-byte aligned, owned by the caller.
+ * Errors: S or H not divisible by degree -> CP_ERR_NOT_DIVISIBLE; otherwise as cp_ring_sim
+ * and cp_ulysses_permute.  Asynchronous on `stream`.
+ */
+CP_API cp_status cp_usp_sim(const void* q, const void* k, const void* v, int degree, const int* chunk_bounds,
+                            int n_chunks, void* out, float* out_lse, int B, int S, int H, int D, float scale,
+                            cp_dtype out_dtype, void* workspace, size_t ws_bytes, void* stream);
+
 /* Size in bytes of the library's static device scratch used by cp_ring_sim_static. */
 #define CP_STATIC_SCRATCH_BYTES (32u << 20)
 
@@ -184,6 +211,30 @@ CP_API cp_status cp_ring_sim_fused(const void* q, const void* k, const void* v, 
 CP_API cp_status cp_ring_sim_static(const void* q, const void* k, const void* v, const int* chunk_bounds,
                              int n_chunks, void* out, float* out_lse, int B, int H, int Sq, int Skv,
                              int D, float scale, cp_dtype out_dtype, void* stream);
+
+/*
+ * cp_ulysses_anything_permute - the Ulysses exchange for shards of unequal size.
+ *
+ * Source: "Context parallelism", section "Ulysses Anything Attention": the sequence length
+ * and the head count need not be divisible by ulysses_degree.  The pages give no layout;
+ * the reading here: sequence shard p holds tokens [seq_bounds[p], seq_bounds[p+1]) of
+ * every head and head shard q holds heads [head_bounds[q], head_bounds[q+1]) of every
+ * token, as even as possible when made by cp_ring_bounds(count, degree, 1, ...) (the
+ * first shards one longer).  Shards are packed back to back:
+ *   sequence-sharded: shard p at element offset B*seq_bounds[p]*H*D, layout [B][S_p][H][D];
+ *   head-sharded:     shard q at element offset B*S*head_bounds[q]*D, layout [B][S][H_q][D].
+ * With equal shards these are exactly the stacked layouts of cp_ulysses_permute.
+ * direction 0: sequence-sharded src -> head-sharded dst; 1: the inverse.  A pure copy,
+ * bit-exact for any element type of elem_bytes (2 or 4) bytes.
+ * seq_bounds, head_bounds: HOST int[degree+1], non-decreasing, from 0 to S and 0 to H;
+ * empty shards are allowed.  src, dst: B*S*H*D elements each, 16-byte aligned, not
+ * overlapping.  degree <= 64.
+ * Errors: bad bounds, overlap -> CP_ERR_INVALID_ARG; degree > 64 or elem_bytes not 2/4
+ * -> CP_ERR_UNSUPPORTED; misaligned -> CP_ERR_MISALIGNED.  Asynchronous on `stream`.
+ */
+CP_API cp_status cp_ulysses_anything_permute(const void* src, void* dst, int degree, const int* seq_bounds,
+                                             const int* head_bounds, int B, int S, int H, int D, int direction,
+                                             int elem_bytes, void* stream);
 
 /*
  * cp_ulysses_permute - the Ulysses all-to-all, simulated as one local copy.

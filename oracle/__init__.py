@@ -17,6 +17,8 @@ message-passing all-to-all.  No function here is "parity unpinned".
 """
 
 from .attention import attention, merge, ring, attention_rows
-from .ulysses import ulysses_fwd, ulysses_inv
+from .ulysses import ulysses_anything_fwd, ulysses_anything_inv, ulysses_fwd, ulysses_inv
+from .usp import usp
 
-__all__ = ["attention", "merge", "ring", "attention_rows", "ulysses_fwd", "ulysses_inv"]
+__all__ = ["attention", "merge", "ring", "attention_rows", "ulysses_fwd", "ulysses_inv", "ulysses_anything_fwd",
+           "ulysses_anything_inv", "usp"]

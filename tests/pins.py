@@ -257,6 +257,22 @@ def pin_chunk_merge_identity(attention, ring):
         assert np.allclose(lse, l2, rtol=0, atol=1e-12), f"split {bounds}: lse"
 
 
+def pin_usp_equals_unsplit(attention, usp):
+    """Unified SP (Ulysses exchange -> ring over each head shard -> inverse exchange) equals
+    unsplit attention (fp64, 1e-12): both all-to-alls are pure data movement and the ring
+    merge is exact, so every degree and block split must give the same O and LSE."""
+    r = _rng(21)
+    B, S, H, D = 2, 12, 4, 3
+    q, k, v = (r.standard_normal((B, S, H, D)) for _ in range(3))
+    o, lse = attention(q, k, v, 0.6)
+    for degree, bounds in ((2, [0, 6, 12]), (4, [0, 5, 5, 12]), (2, [0, 12]), (1, [0, 4, 8, 12]), (4, [0, 1, 12])):
+        shard = lambda x: x.reshape(B, degree, S // degree, H, D).transpose(1, 0, 2, 3, 4)
+        o_sh, l2 = usp(shard(q), shard(k), shard(v), degree, 0.6, bounds)
+        o2 = np.asarray(o_sh).transpose(1, 0, 2, 3, 4).reshape(B, S, H, D)
+        assert np.allclose(o, o2, rtol=0, atol=1e-12), f"usp {degree} x {bounds}: o"
+        assert np.allclose(lse, l2, rtol=0, atol=1e-12), f"usp {degree} x {bounds}: lse"
+
+
 # --------------------------------------------------------------------------- Ulysses
 
 
@@ -319,3 +335,53 @@ def pin_ulysses_golden(ulysses_fwd):
     for rank, tok, *vals in rows:
         assert list(dst[rank, 0, tok, :, 0]) == vals, f"golden rank {rank} token {tok}"
     assert len(rows) == P * S
+
+
+# --------------------------------------------------------------------------- Ulysses Anything
+
+def _near_even(count, parts):
+    """Bounds of ``parts`` shards as even as possible, the first ``count % parts`` one longer."""
+    base, extra = divmod(count, parts)
+    b = [0]
+    for p in range(parts):
+        b.append(b[-1] + base + (1 if p < extra else 0))
+    return b
+
+
+ANYTHING_CASES = [
+    # (S, H, seq_bounds, head_bounds)
+    (7, 5, [0, 3, 5, 7], [0, 2, 4, 5]),                  # both uneven, P = 3
+    (10, 3, [0, 3, 6, 8, 10], [0, 1, 2, 3, 3]),          # an empty head group, P = 4
+    (9, 6, [0, 0, 4, 9], [0, 2, 4, 6]),                  # an empty sequence shard
+    (13, 24, _near_even(13, 5), _near_even(24, 5)),      # heads not divisible by 5
+    (17, 4, _near_even(17, 4), _near_even(4, 4)),        # FLUX-1008-like: tokens not divisible by 4
+]
+
+
+def pin_anything_origin(ulysses_anything_fwd, ulysses_anything_inv):
+    """Every input value encodes its origin (b, s, h, d) exactly in fp64; after the exchange,
+    position (b, s, j, d) of head shard q must hold the code of (b, s, head_bounds[q] + j, d),
+    computed here by formula, and the inverse must restore every sequence shard."""
+    B, D = 2, 3
+    code = lambda b, s, h, d: ((b * 100.0 + s) * 100.0 + h) * 10.0 + d
+    for S, H, sb, hb in ANYTHING_CASES:
+        X = np.fromfunction(code, (B, S, H, D))
+        shards = [X[:, sb[p]:sb[p + 1]] for p in range(len(sb) - 1)]
+        out = ulysses_anything_fwd(shards, sb, hb)
+        for q in range(len(hb) - 1):
+            want = np.fromfunction(lambda b, s, j, d: code(b, s, hb[q] + j, d), (B, S, hb[q + 1] - hb[q], D))
+            assert np.asarray(out[q]).shape == want.shape and np.array_equal(np.asarray(out[q]), want), (S, H, q)
+        back = ulysses_anything_inv(out, sb, hb)
+        for p in range(len(sb) - 1):
+            assert np.array_equal(np.asarray(back[p]), shards[p]), (S, H, p)
+
+
+def pin_anything_reduces_to_even(ulysses_anything_fwd, ulysses_fwd):
+    """With equal shards the Anything exchange is the (golden-pinned) even exchange."""
+    r = _rng(23)
+    P, B, S, H, D = 4, 2, 8, 8, 2
+    stacked = r.standard_normal((P, B, S // P, H, D))
+    even = ulysses_fwd(stacked, P)
+    any_ = ulysses_anything_fwd([stacked[p] for p in range(P)], _near_even(S, P), _near_even(H, P))
+    for q in range(P):
+        assert np.array_equal(np.asarray(any_[q]), np.asarray(even[q]))

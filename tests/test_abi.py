@@ -118,6 +118,46 @@ def test_workspace_size(lib):
     assert binding.ring_workspace_size(n, B, H, S, D) == want
 
 
+def test_usp_sim_checks_before_launch(lib):
+    p = ctypes.c_void_p(1 << 20)
+    # (degree, S, H, bounds, ws_bytes, want); pointers are fake, every check precedes CUDA
+    cases = [
+        (3, 16, 6, (0, 16), 1 << 30, I.CP_ERR_NOT_DIVISIBLE),   # S % degree
+        (4, 16, 6, (0, 16), 1 << 30, I.CP_ERR_NOT_DIVISIBLE),   # H % degree
+        (2, 16, 4, (0, 9, 15), 1 << 30, I.CP_ERR_INVALID_ARG),  # bounds do not span [0, S]
+        (2, 16, 4, (0, 8, 16), 100, I.CP_ERR_INVALID_ARG),      # workspace too small
+        (0, 16, 4, (0, 16), 1 << 30, I.CP_ERR_INVALID_ARG),     # degree < 1
+    ]
+    for degree, S, H, b, ws, want in cases:
+        st = lib.cp_usp_sim(p, p, p, degree, _bounds(*b), len(b) - 1, p, None, 1, S, H, 64, 0.1, 0, p, ws, None)
+        assert st == want, (degree, S, H, b, ws, st)
+
+
+def test_ulysses_anything_checks_before_launch(lib):
+    p = ctypes.c_void_p(1 << 20)
+    q = ctypes.c_void_p((1 << 20) + 8)
+    ok_s, ok_h = _bounds(0, 3, 5, 7), _bounds(0, 2, 4, 5)
+    call = lambda src, dst, deg, sb, hb, eb=2, direction=0: lib.cp_ulysses_anything_permute(
+        src, dst, deg, sb, hb, 1, 7, 5, 64, direction, eb, None)
+    assert call(p, p, 3, _bounds(0, 3, 5, 6), ok_h) == I.CP_ERR_INVALID_ARG   # does not end at S
+    assert call(p, p, 3, ok_s, _bounds(0, 3, 2, 5)) == I.CP_ERR_INVALID_ARG   # decreasing
+    assert call(p, p, 3, ok_s, ok_h, eb=8) == I.CP_ERR_UNSUPPORTED
+    assert call(p, p, 3, ok_s, ok_h, direction=2) == I.CP_ERR_INVALID_ARG
+    assert call(p, p, 3, ok_s, ok_h) == I.CP_ERR_INVALID_ARG                  # src and dst overlap
+    assert call(p, q, 3, ok_s, ok_h) == I.CP_ERR_MISALIGNED
+    big = list(range(66))
+    assert lib.cp_ulysses_anything_permute(p, p, 65, _bounds(*big), _bounds(*big), 1, 65, 65, 64, 0, 2,
+                                           None) == I.CP_ERR_UNSUPPORTED        # degree > 64
+
+
+def test_usp_workspace_size():
+    U, n, B, S, H, D = 2, 4, 1, 4608, 24, 128
+    elems = B * S * H * D
+    ring = binding.ring_workspace_size(n, U * B, H // U, S, D)
+    assert binding.usp_workspace_size(U, n, B, S, H, D) == 3 * elems * 2 + elems * 2 + B * H * S * 4 + ring
+    assert binding.usp_workspace_size(5, n, B, S, H, D) == 0  # 24 heads are not divisible by 5
+
+
 def test_ring_bounds():
     assert binding.ring_bounds(4608, 8) == [576 * i for i in range(9)]
     assert binding.ring_bounds(4173, 3, anything=True) == [0, 1391, 2782, 4173]

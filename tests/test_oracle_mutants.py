@@ -18,6 +18,9 @@ ORACLE = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))
 def _load_mutant(fname, old, new):
     src = open(os.path.join(ORACLE, fname)).read()
     assert src.count(old) == 1, f"mutation anchor not unique/found: {old!r}"
+    # The mutant runs outside the package: its relative imports take the (unmutated) oracle.
+    src = src.replace("from .attention import", "from oracle.attention import").replace(
+        "from .ulysses import", "from oracle.ulysses import")
     ns = {"__name__": "oracle_mutant"}
     exec(compile(src.replace(old, new), f"<mutant {fname}>", "exec"), ns)
     return ns
@@ -64,6 +67,22 @@ ULYSSES_MUTANTS = [
 ]
 
 
+ANYTHING_MUTANTS = [
+    ("owner by average shard size", "owner = _owner(seq_bounds, s)", "owner = min(s // -(-S // P), P - 1)"),
+    ("head groups by floor split", "hq0, hq1 = int(head_bounds[q]), int(head_bounds[q + 1])\n        shape = (B, S, hq1 - hq0, D)",
+     "hq0, hq1 = q * H // P, (q + 1) * H // P\n        shape = (B, S, hq1 - hq0, D)"),
+    ("local index from an even stride", "s - int(seq_bounds[owner])", "s - owner * (S // P)"),
+]
+
+USP_MUTANTS = [
+    ("LSE head groups reversed", "lse = np.concatenate(lses, axis=1)", "lse = np.concatenate(lses[::-1], axis=1)"),
+    ("K/V of the first head group everywhere", "o_p, lse_p, _, _ = ring(qh[p], kh[p], vh[p], scale, chunk_bounds)",
+     "o_p, lse_p, _, _ = ring(qh[p], kh[0], vh[0], scale, chunk_bounds)"),
+    ("keys used as values", "o_p, lse_p, _, _ = ring(qh[p], kh[p], vh[p], scale, chunk_bounds)",
+     "o_p, lse_p, _, _ = ring(qh[p], kh[p], kh[p], scale, chunk_bounds)"),
+]
+
+
 @pytest.mark.parametrize("name,old,new", ATTN_MUTANTS, ids=[m[0] for m in ATTN_MUTANTS])
 def test_attention_mutant_is_caught(name, old, new):
     ns = _load_mutant("attention.py", old, new)
@@ -86,4 +105,22 @@ def test_ulysses_mutant_is_caught(name, old, new):
     ns = _load_mutant("ulysses.py", old, new)
     checks = [lambda: pins.pin_ulysses_messages(ns["ulysses_fwd"]), lambda: pins.pin_ulysses_golden(ns["ulysses_fwd"]),
               lambda: pins.pin_ulysses_roundtrip(ns["ulysses_fwd"], ns["ulysses_inv"])]
+    assert any(_fails(c) for c in checks), f"mutant '{name}' passed every pin"
+
+
+@pytest.mark.parametrize("name,old,new", USP_MUTANTS, ids=[m[0] for m in USP_MUTANTS])
+def test_usp_mutant_is_caught(name, old, new):
+    import oracle
+
+    ns = _load_mutant("usp.py", old, new)
+    assert _fails(lambda: pins.pin_usp_equals_unsplit(oracle.attention, ns["usp"])), f"mutant '{name}' passed"
+
+
+@pytest.mark.parametrize("name,old,new", ANYTHING_MUTANTS, ids=[m[0] for m in ANYTHING_MUTANTS])
+def test_ulysses_anything_mutant_is_caught(name, old, new):
+    import oracle
+
+    ns = _load_mutant("ulysses.py", old, new)
+    checks = [lambda: pins.pin_anything_origin(ns["ulysses_anything_fwd"], oracle.ulysses_anything_inv),
+              lambda: pins.pin_anything_reduces_to_even(ns["ulysses_anything_fwd"], oracle.ulysses_fwd)]
     assert any(_fails(c) for c in checks), f"mutant '{name}' passed every pin"

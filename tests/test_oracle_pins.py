@@ -22,6 +22,18 @@ def test_chunk_merge_identity():
     pins.pin_chunk_merge_identity(oracle.attention, oracle.ring)
 
 
+def test_usp_equals_unsplit():
+    pins.pin_usp_equals_unsplit(oracle.attention, oracle.usp)
+
+
+def test_ulysses_anything_origin():
+    pins.pin_anything_origin(oracle.ulysses_anything_fwd, oracle.ulysses_anything_inv)
+
+
+def test_ulysses_anything_reduces_to_even():
+    pins.pin_anything_reduces_to_even(oracle.ulysses_anything_fwd, oracle.ulysses_fwd)
+
+
 def test_ulysses_message_passing():
     pins.pin_ulysses_messages(oracle.ulysses_fwd)
 
