@@ -61,11 +61,13 @@ constexpr int kVProducerWarp = 10; // V loads
 constexpr int kPvWarp = 11;        // P.V issuer
 constexpr int kEpilogueWarp0 = 12;
 // setmaxnreg split of the 128 x 512 launch budget: softmax (8 warps), control (warps 8-11),
-// epilogue (warps 12-15).
-constexpr int kSoftmaxRegs = 152;
-constexpr int kControlRegs = 96;
-constexpr int kEpilogueRegs = 112;
+// epilogue (warps 12-15, enough to hold a whole O row: it releases O before storing it).
+constexpr int kSoftmaxRegs = 136;
+constexpr int kControlRegs = 48;
+constexpr int kEpilogueRegs = 192;
 static_assert(2 * kSoftmaxRegs + kControlRegs + kEpilogueRegs == 4 * 128, "register split must use the launch budget");
+static_assert(kSoftmaxRegs >= 128 && kEpilogueRegs >= 128 && kControlRegs <= 128,
+              "softmax and epilogue warpgroups grow (setmaxnreg.inc), the control warps shrink");
 constexpr int kTmemCols = 512;
 constexpr int kTmemO = 256;        // first O column; O_k at kTmemO + 128 k
 constexpr int kMaxChunks = 64;
@@ -697,24 +699,36 @@ __device__ __forceinline__ void attn_epilogue(const AttnParams& p, uint8_t* smem
       const float c0f = w0 * inv, c1f = w1 * inv;
       const size_t o_off = static_cast<size_t>(c) * p.out_chunk_stride +
                            ((static_cast<size_t>(uc.b) * p.Sq + s_row) * p.H + uc.h) * D;
-#pragma unroll 1
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t r[32];
-        tmem_ld32(to0 + cc * 32, r);
-        if (__any_sync(0xffffffffu, has1)) {
+      // Read the whole merged O row into registers and release O before storing it: every
+      // CTA reaches its block ends at about the same time, so a segment's stores run into
+      // HBM bandwidth, and the next segment's first P.V must not wait for them.
+      uint32_t r[D];
+      if constexpr (D == 128)
+        tmem_ld128(to0, r);
+      else
+        tmem_ld64(to0, r);
+      const bool any1 = __any_sync(0xffffffffu, has1);
+      if (any1) {
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t r1[32];
           tmem_ld32(to1 + cc * 32, r1);
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            r[i] = __float_as_uint(fmaf(__uint_as_float(r[i]), c0f, has1 ? __uint_as_float(r1[i]) * c1f : 0.f));
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * c0f);
+            r[cc * 32 + i] = __float_as_uint(
+                fmaf(__uint_as_float(r[cc * 32 + i]), c0f, has1 ? __uint_as_float(r1[i]) * c1f : 0.f));
         }
-        if (row_ok) store_row<D>(p, o_off, r, cc);
       }
       tc_fence_before();
       warp_arrive(bars + kOFree);
+      if (!any1) {
+#pragma unroll
+        for (int i = 0; i < D; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * c0f);
+      }
+      if (row_ok) {
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) store_row<D>(p, o_off, *reinterpret_cast<const uint32_t(*)[32]>(r + cc * 32), cc);
+      }
       if (row_ok && p.lse)
         p.lse[static_cast<size_t>(c) * p.lse_chunk_stride + (static_cast<size_t>(uc.b) * p.H + uc.h) * p.Sq +
               s_row] = (mx + log2f(lsum)) * 0.69314718055994530942f;
@@ -774,7 +788,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   // Producer and MMA roles run on lane 0 of their warp; the other lanes wait at the
   // __syncwarp so that each warp is converged again for the teardown below.
   if (warp >= kEpilogueWarp0) {
-    regs_decrease<kEpilogueRegs>();
+    regs_increase<kEpilogueRegs>();
     attn_epilogue<D>(p, smem, bars, tmem, abort_flag);
   } else if (warp >= 8) {
     regs_decrease<kControlRegs>();
