@@ -37,12 +37,12 @@ UNIT = "TFLOP/s"
 
 # DRAM traffic of the timed attention launch (8 ring blocks, FLUX B1), from one ncu capture
 # of the same kernel on the B2 shape (profiles/attn_fwd_sm100__flux_b2_ring8.md):
-# dram__bytes_read.sum + dram__bytes_write.sum = 185.78 + 861.37 MB, halved to one B1 launch
+# dram__bytes_read.sum + dram__bytes_write.sum = 185.87 + 862.32 MB, halved to one B1 launch
 # (the B1 launch processes half the units; Q/K/V reads and partial writes scale with them).
 # It describes only the kernel source it was captured on, identified by its SHA-256.
 ATTN_TRAFFIC = {
-    "kernel_sha256": "8f5d0b897bd65637f466a9f0c3b0ae5212c8f95804f07fa503d6956c61afcf98",
-    "bytes_per_launch": (185_780_224 + 861_372_160) // 2,
+    "kernel_sha256": "95637b860ddd7bd742d9ce1154c2e05af9c4e26427313ba40c26b59d77f23e4f",
+    "bytes_per_launch": (185_868_032 + 862_317_568) // 2,
 }
 
 
