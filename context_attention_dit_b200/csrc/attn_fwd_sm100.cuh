@@ -602,7 +602,6 @@ __device__ __forceinline__ void attn_softmax(const AttnParams& p, uint8_t* smem,
   const uint32_t to = tmem + lanes + kTmemO + kh * 128;  // O_k
   float2* stat = reinterpret_cast<float2*>(smem + L::kStat) + kh * 2 * kBM;
   const float sl2 = p.scale_log2;
-  const int gbar = kBarSoftmax0 + kh;
   uint32_t g = 0;     // tiles seen
   uint32_t nch = 0;   // segments finished
   bool alive = true;  // false once a wait of this thread gave up
@@ -628,7 +627,7 @@ __device__ __forceinline__ void attn_softmax(const AttnParams& p, uint8_t* smem,
       for (int j = 0; j < n_kv; ++j, ++g) {
         const Tile t = make_tile(p, c, j);
         const int sb = g & 1;
-        if (!group_wait(bars + kQkDone + sb, (g >> 1) & 1, gbar, alive, abort_flag, p.status)) return;
+        if (!warp_wait(bars + kQkDone + sb, (g >> 1) & 1, abort_flag, p.status) || !alive) return;
         tc_fence_after();
         const int vh = half_valid(t.valid(), kh);
         if (vh > 0) {
@@ -650,7 +649,7 @@ __device__ __forceinline__ void attn_softmax(const AttnParams& p, uint8_t* smem,
       // segment (it releases O only after reading that segment's stats): without this
       // wait, one-tile segments let this warpgroup run two stat_ready phases ahead of the
       // epilogue, which a parity wait cannot tell apart.
-      if (nch > 0 && !group_wait(bars + kOFree, (nch - 1) & 1, gbar, alive, abort_flag, p.status)) return;
+      if (nch > 0 && (!warp_wait(bars + kOFree, (nch - 1) & 1, abort_flag, p.status) || !alive)) return;
       stat[(nch & 1) * kBM + row] = make_float2(m, l);
       warp_arrive(bars + kStatReady);
       ++nch;

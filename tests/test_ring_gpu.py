@@ -186,3 +186,23 @@ def test_fused_flux_ring8_and_uneven():
     o_ref2, lse_ref2 = workload_oracle("uneven_s4173_ring3")
     o2, lse2 = binding.ring_sim_fused(*cuda(q2, k2, v2), bounds_from_sizes(w2.splits[1]), scale=w2.scale)
     assert_attn_close(o2, lse2, o_ref2, lse_ref2, "fused uneven 1392/1391/1390")
+
+
+def test_bench_step_launch_configuration():
+    """The hot path exactly as bench.py times it on FLUX: the Ulysses-8 exchange of Q, K, V
+    in one launch, ring-8 attention over the head-sharded tensors (batch 8, 3 heads) in one
+    launch, the LSE merge, the inverse exchange of O.  Every element against fp64."""
+    w, (q, k, v) = workload_inputs("flux_1024_ring8_ulysses8")
+    o_ref, lse_ref = workload_oracle("flux_1024_ring1")  # same inputs (seed, shape, QK-norm)
+    P, B, S, H, D = 8, w.B, w.S, w.H, w.D
+    xs = [t.reshape(B, P, S // P, H, D).permute(1, 0, 2, 3, 4).contiguous().cuda() for t in (q, k, v)]
+    ys = binding.ulysses_permute_n(xs, P, 0)
+    view = lambda t: t.view(P * B, S, H // P, D)
+    parts, lses = binding.attn_fwd_blocks(view(ys[0]), view(ys[1]), view(ys[2]), even_bounds(S, 8), scale=w.scale)
+    o_h, lse_h = binding.attn_merge(parts, lses)
+    o_seq = binding.ulysses_permute(o_h.view(P, B, S, H // P, D), P, 1)
+    torch.cuda.synchronize()
+    assert binding.last_device_status() == 0
+    o = o_seq.permute(1, 0, 2, 3, 4).reshape(B, S, H, D)
+    lse = lse_h.view(P, B, H // P, S).permute(1, 0, 2, 3).reshape(B, H, S)  # head group p = heads 3p..3p+2
+    assert_attn_close(o, lse, o_ref, lse_ref, "bench step (FLUX Ulysses-8 x ring-8)")
