@@ -203,12 +203,12 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, ok);
 }
 
-// Named barriers (id 0 is __syncthreads): one per softmax warpgroup and the epilogue.
-constexpr int kBarSoftmax0 = 1;
-constexpr int kBarEpilogue = 3;
+// Named barrier of the epilogue warpgroup (id 0 is __syncthreads).
+constexpr int kBarEpilogue = 1;
 
 // A 128-thread warpgroup waits for `bar`: only its first warp polls (fewer mbarrier polls
-// in the MIO queue), the others park at named barrier `id`.  `alive` carries an earlier
+// in the MIO queue, for a group that waits most of the time), the others park at named
+// barrier `id`.  `alive` carries an earlier
 // failure of this thread into the decision, so that every warp of the group leaves
 // together: a named barrier that one warp never reaches would never complete.
 __device__ __forceinline__ bool group_wait(uint64_t* bar, uint32_t parity, int id, bool alive,
