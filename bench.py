@@ -37,12 +37,12 @@ UNIT = "TFLOP/s"
 
 # DRAM traffic of the timed attention launch (8 ring blocks, FLUX B1), from one ncu capture
 # of the same kernel on the B2 shape (profiles/attn_fwd_sm100__flux_b2_ring8.md):
-# dram__bytes_read.sum + dram__bytes_write.sum = 185.87 + 862.32 MB, halved to one B1 launch
+# dram__bytes_read.sum + dram__bytes_write.sum = 185.73 + 862.05 MB, halved to one B1 launch
 # (the B1 launch processes half the units; Q/K/V reads and partial writes scale with them).
 # It describes only the kernel source it was captured on, identified by its SHA-256.
 ATTN_TRAFFIC = {
-    "kernel_sha256": "95637b860ddd7bd742d9ce1154c2e05af9c4e26427313ba40c26b59d77f23e4f",
-    "bytes_per_launch": (185_868_032 + 862_317_568) // 2,
+    "kernel_sha256": "865bd87726044ea2ec385acff9c4d10946c62fe02430734494319448dadfcea7",
+    "bytes_per_launch": (185_726_976 + 862_048_000) // 2,
 }
 
 
@@ -191,12 +191,13 @@ def run_ours(args):
     yq, yk, yv = (torch.empty((P, B, S, Hp, D), dtype=torch.bfloat16, device=dev) for _ in range(3))
     o_h = torch.empty((Bp, S, Hp, D), dtype=torch.bfloat16, device=dev)
     lse_h = torch.empty((Bp, Hp, S), dtype=torch.float32, device=dev)
+    lse_full = torch.empty((B, H, S), dtype=torch.float32, device=dev)
     o_seq = torch.empty((P, B, S // P, H, D), dtype=torch.bfloat16, device=dev)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
     scale = w.scale
     flop = w.flop
-    launches_per_step = 1 + 2 + 1  # permute (Q,K,V), attention, merge, inverse permute
+    launches_per_step = 1 + 1 + 1  # exchange of Q, K, V; attention; merge fused with the inverse exchange
 
     def step(evs=None, x=None, out=None):
         x = x or (xq, xk, xv)
@@ -210,12 +211,11 @@ def run_ours(args):
         binding.attn_fwd_blocks(view(yq), view(yk), view(yv), bounds, scale=scale, partials=parts, lses=lses)
         if evs:
             evs[2].record()
-        binding.attn_merge(parts, lses, out=o_h, out_lse=lse_h)
+        # The LSE merge writes each merged row straight to its sequence-sharded position: the
+        # merge and the second all-to-all in one pass (cp_attn_merge_ulysses).
+        binding.attn_merge_ulysses(parts, lses, P, out=out, out_lse=lse_full)
         if evs:
             evs[3].record()
-        binding.ulysses_permute(o_h.view(P, B, S, Hp, D), P, 1, dst=out)
-        if evs:
-            evs[4].record()
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -225,7 +225,7 @@ def run_ours(args):
 
     clocks = ClockSampler(local)
     clocks.start()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -240,11 +240,10 @@ def run_ours(args):
     clocks.stop()
     assert binding.last_device_status() == 0, "device status not OK after timed region"
 
-    step_ms = [e[0].elapsed_time(e[4]) for e in evs]
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
     perm_ms = [e[0].elapsed_time(e[1]) for e in evs]
     attn_ms = [e[1].elapsed_time(e[2]) for e in evs]
     merge_ms = [e[2].elapsed_time(e[3]) for e in evs]
-    inv_ms = [e[3].elapsed_time(e[4]) for e in evs]
     total_ms = reduce_max(sum(step_ms), dev)
 
     # Single-block attention (the FLUX ring-1 case) timed on its own.
@@ -370,7 +369,6 @@ def run_ours(args):
         rows = Bp * Hp * S
         merge_bytes = n_blocks * rows * (4 * D + 4) + rows * (2 * D + 4)
         perm_bytes = 3 * 2 * B * S * H * D * 2
-        inv_bytes = 2 * B * S * H * D * 2
         part_bytes = n_blocks * rows * (4 * D + 4)
         line = {
             "metric": METRIC,
@@ -416,12 +414,10 @@ def run_ours(args):
                 "ring8_fused_ms": round(fused_ms, 4),
                 "ring8_fused_tflops": round(flop / (fused_ms * 1e-3) / 1e12, 2),
                 "attn_ring8_partial_bytes": part_bytes,
-                "merge_ms": round(statistics.mean(merge_ms), 4),
-                "merge_gbs": round(merge_bytes / (statistics.mean(merge_ms) * 1e-3) / 1e9, 1),
+                "merge_inverse_exchange_ms": round(statistics.mean(merge_ms), 4),
+                "merge_inverse_exchange_gbs": round(merge_bytes / (statistics.mean(merge_ms) * 1e-3) / 1e9, 1),
                 "permute_qkv_ms": round(statistics.mean(perm_ms), 4),
                 "permute_qkv_gbs": round(perm_bytes / (statistics.mean(perm_ms) * 1e-3) / 1e9, 1),
-                "permute_inv_ms": round(statistics.mean(inv_ms), 4),
-                "permute_inv_gbs": round(inv_bytes / (statistics.mean(inv_ms) * 1e-3) / 1e9, 1),
                 "hbm_peak_gbs": peaks["hbm_gbs"],
                 **usp,
                 "anything_permute_flux1008_p4_ms": round(any_ms, 4),
@@ -545,10 +541,10 @@ def run_profile_case(args):
             binding.attn_fwd(q, k, v)
         elif case == "attn_ring8":
             binding.attn_fwd_blocks(q, k, v, bounds)
-        elif case == "merge":
-            parts = torch.randn(8, B, S, H, D, device="cuda")
-            lses = torch.randn(8, B, H, S, device="cuda")
-            binding.attn_merge(parts, lses)
+        elif case == "merge":  # the step's merge: head-shard partials, fused with the inverse exchange
+            parts = torch.randn(8, P * B, S, H // P, D, device="cuda")
+            lses = torch.randn(8, P * B, H // P, S, device="cuda")
+            binding.attn_merge_ulysses(parts, lses, P)
         elif case == "permute":
             xs = [t.view(B, P, S // P, H, D).permute(1, 0, 2, 3, 4).contiguous() for t in (q, k, v)]
             ys = binding.ulysses_permute_n(xs, P, 0)

@@ -35,7 +35,7 @@ EXPORTS = (
     "cp_attn_fwd", "cp_attn_fwd_blocks", "cp_attn_merge", "cp_ring_sim_workspace_size", "cp_ring_sim",
     "cp_ring_sim_fused", "cp_ring_sim_static", "cp_ulysses_permute", "cp_ulysses_permute_n", "cp_ring_bounds",
     "cp_debug_set_fault", "cp_last_device_status", "cp_status_string", "cp_version", "cp_usp_sim_workspace_size",
-    "cp_usp_sim", "cp_ulysses_anything_permute",
+    "cp_usp_sim", "cp_ulysses_anything_permute", "cp_attn_merge_ulysses",
 )
 
 _lib = None
@@ -60,6 +60,7 @@ def load() -> ctypes.CDLL:
     lib.cp_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
     lib.cp_attn_fwd_blocks.argtypes = [vp, vp, vp, ip, i, vp, vp, i, i, i, i, i, f, vp]
     lib.cp_attn_merge.argtypes = [vp, vp, i, vp, vp, i, i, i, i, i, vp]
+    lib.cp_attn_merge_ulysses.argtypes = [vp, vp, i, vp, vp, i, i, i, i, i, i, vp]
     lib.cp_ring_sim_workspace_size.argtypes = [i, i, i, i, i]
     lib.cp_ring_sim_workspace_size.restype = sz
     lib.cp_ring_sim.argtypes = [vp, vp, vp, ip, i, vp, vp, i, i, i, i, i, f, i, vp, sz, vp]
@@ -192,6 +193,30 @@ def attn_merge(partials, lses, out_dtype=torch.bfloat16, out=None, out_lse=None)
 
 def ring_workspace_size(n_chunks: int, B: int, H: int, Sq: int, D: int) -> int:
     return int(load().cp_ring_sim_workspace_size(n_chunks, B, H, Sq, D))
+
+
+def attn_merge_ulysses(partials, lses, degree: int, out_dtype=torch.bfloat16, out=None, out_lse=None):
+    """Merge of Ulysses head-shard partials ``[n, degree*B, S, H/degree, D]`` (LSEs ``[n,
+    degree*B, H/degree, S]``) fused with the inverse exchange: returns ``(out [degree, B,
+    S/degree, H, D], lse [B, H, S])``, identical to :func:`attn_merge` then the inverse
+    :func:`ulysses_permute`."""
+    if partials.dtype != torch.float32 or lses.dtype != torch.float32:
+        raise ValueError("partials and lses must be float32")
+    if not (partials.is_cuda and lses.is_cuda and partials.is_contiguous() and lses.is_contiguous()):
+        raise ValueError("partials and lses must be contiguous CUDA tensors")
+    n, PB, S, Hp, D = partials.shape
+    if PB % degree != 0 or lses.shape != (n, PB, Hp, S):
+        raise ValueError(f"incompatible shapes partials{tuple(partials.shape)} lses{tuple(lses.shape)}")
+    B, H = PB // degree, Hp * degree
+    code = _out_code(out_dtype)
+    if out is None:
+        out = torch.empty((degree, B, S // degree, H, D), dtype=out_dtype, device=partials.device)
+    if out_lse is None:
+        out_lse = torch.empty((B, H, S), dtype=torch.float32, device=partials.device)
+    st = load().cp_attn_merge_ulysses(_ptr(partials), _ptr(lses), n, _ptr(out), _ptr(out_lse), degree, B, S, H, D, code,
+                                      ctypes.c_void_p(_stream(partials)))
+    _check(st, "cp_attn_merge_ulysses")
+    return out, out_lse
 
 
 def ring_sim(q, k, v, chunk_bounds: Sequence[int], scale: Optional[float] = None, out_dtype=torch.bfloat16,

@@ -173,7 +173,7 @@ cp_status launch_attn(const void* q, const void* k, const void* v, const int* bo
 }
 
 cp_status launch_merge(const float* partials, const float* lses, int n, void* out, float* out_lse, int B, int H,
-                       int Sq, int D, cp_dtype out_dtype, cudaStream_t stream) {
+                       int Sq, int D, cp_dtype out_dtype, cudaStream_t stream, int ulysses_p = 0, int ulysses_b = 0) {
   const long long rows = static_cast<long long>(B) * H * Sq;
   const long long part_stride = rows * D;
   const long long lse_stride = rows;
@@ -184,20 +184,21 @@ cp_status launch_merge(const float* partials, const float* lses, int n, void* ou
   const size_t smem = static_cast<size_t>(n) * H * ST * sizeof(float);
   if (smem > 48 * 1024) return CP_ERR_UNSUPPORTED;
   const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(B));
-  if (D == 128) {
-    if (out_dtype == CP_BF16)
-      lse_merge_kernel<128, true><<<grid, kMergeThreads, smem, stream>>>(partials, lses, n, out, out_lse, H, Sq, ST,
-                                                                         part_stride, lse_stride);
+  auto launch = [&](auto kernel) {
+    kernel<<<grid, kMergeThreads, smem, stream>>>(partials, lses, n, out, out_lse, H, Sq, ST, part_stride, lse_stride,
+                                                  ulysses_p, ulysses_b);
+  };
+  const bool bf16 = out_dtype == CP_BF16;
+  if (ulysses_p > 0) {
+    if (D == 128)
+      bf16 ? launch(lse_merge_kernel<128, true, true>) : launch(lse_merge_kernel<128, false, true>);
     else
-      lse_merge_kernel<128, false><<<grid, kMergeThreads, smem, stream>>>(partials, lses, n, out, out_lse, H, Sq, ST,
-                                                                          part_stride, lse_stride);
+      bf16 ? launch(lse_merge_kernel<64, true, true>) : launch(lse_merge_kernel<64, false, true>);
   } else {
-    if (out_dtype == CP_BF16)
-      lse_merge_kernel<64, true><<<grid, kMergeThreads, smem, stream>>>(partials, lses, n, out, out_lse, H, Sq, ST,
-                                                                        part_stride, lse_stride);
+    if (D == 128)
+      bf16 ? launch(lse_merge_kernel<128, true, false>) : launch(lse_merge_kernel<128, false, false>);
     else
-      lse_merge_kernel<64, false><<<grid, kMergeThreads, smem, stream>>>(partials, lses, n, out, out_lse, H, Sq, ST,
-                                                                         part_stride, lse_stride);
+      bf16 ? launch(lse_merge_kernel<64, true, false>) : launch(lse_merge_kernel<64, false, false>);
   }
   return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
 }
@@ -464,6 +465,22 @@ cp_status cp_ulysses_permute_n(const void* const* srcs, void* const* dsts, int n
   else
     launch(uint16_t{});
   return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+}
+
+cp_status cp_attn_merge_ulysses(const float* partials, const float* lses, int n_chunks, void* out, float* out_lse,
+                                int degree, int B, int S, int H, int D, cp_dtype out_dtype, void* stream) {
+  if (degree < 1 || B < 0 || S < 0 || H < 0) return CP_ERR_INVALID_ARG;
+  if (S % degree != 0 || H % degree != 0) return CP_ERR_NOT_DIVISIBLE;
+  if (n_chunks < 1 || n_chunks > CP_MAX_CHUNKS) return n_chunks < 1 ? CP_ERR_INVALID_ARG : CP_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128) return CP_ERR_UNSUPPORTED;
+  if (out_dtype != CP_BF16 && out_dtype != CP_F32) return CP_ERR_INVALID_ARG;
+  if (B == 0 || H == 0 || S == 0) return CP_OK;
+  if (!partials || !lses || !out) return CP_ERR_INVALID_ARG;
+  if (!aligned16(partials) || !aligned16(lses) || !aligned16(out) || (out_lse && !aligned16(out_lse)))
+    return CP_ERR_MISALIGNED;
+  if (static_cast<long long>(degree) * B > 65535) return CP_ERR_UNSUPPORTED;
+  return launch_merge(partials, lses, n_chunks, out, out_lse, degree * B, H / degree, S, D, out_dtype,
+                      static_cast<cudaStream_t>(stream), degree, B);
 }
 
 cp_status cp_ulysses_anything_permute(const void* src, void* dst, int degree, const int* seq_bounds,

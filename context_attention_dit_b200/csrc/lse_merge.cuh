@@ -24,10 +24,15 @@ namespace cpattn {
 
 constexpr int kMergeThreads = 256;
 
-template <int D, bool kOutBf16>
+// kUlysses: the partials are those of attention on Ulysses head shards (batch P*Bs, H heads
+// per shard, shard p = heads [p*H, (p+1)*H) of P*H), and the merged output goes straight to
+// the sequence-sharded layout of the inverse exchange, [P][Bs][Sq/P][P*H][D] (the merge and
+// the second all-to-all of "Ulysses Attention" in one pass), with the LSE as [Bs][P*H][Sq].
+template <int D, bool kOutBf16, bool kUlysses>
 __global__ void __launch_bounds__(kMergeThreads)
     lse_merge_kernel(const float* __restrict__ partials, const float* __restrict__ lses, int n, void* __restrict__ out,
-                     float* __restrict__ out_lse, int H, int Sq, int ST, long long part_stride, long long lse_stride) {
+                     float* __restrict__ out_lse, int H, int Sq, int ST, long long part_stride, long long lse_stride,
+                     int P, int Bs) {
   constexpr int kVec = D / 32;  // floats per lane: 4 (D=128) or 2 (D=64)
   constexpr float kLog2e = 1.4426950408889634f;
   constexpr float kLn2 = 0.69314718055994530942f;
@@ -57,15 +62,24 @@ __global__ void __launch_bounds__(kMergeThreads)
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     const long long row = (static_cast<long long>(b) * Sq + s) * H + h;  // BSHD row
     const long long eoff = row * D + lane * kVec;
-    const long long lrow = (static_cast<long long>(b) * H + h) * Sq + s;  // [B][H][Sq]
+    long long ooff = eoff;                                                 // output element
+    long long lrow = (static_cast<long long>(b) * H + h) * Sq + s;        // [B][H][Sq]
+    if (kUlysses) {
+      const int p = b / Bs, bs = b - (b / Bs) * Bs;  // head shard, batch
+      const int Sp = Sq / P;
+      const int ps = s / Sp, sl = s - (s / Sp) * Sp;  // sequence shard, token within it
+      ooff = (((static_cast<long long>(ps) * Bs + bs) * Sp + sl) * (static_cast<long long>(P) * H) + p * H + h) * D +
+             lane * kVec;
+      lrow = (static_cast<long long>(bs) * P * H + p * H + h) * Sq + s;
+    }
     if (M == -INFINITY) {  // every block empty
       if (kOutBf16) {
         if (kVec == 4)
-          *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out) + eoff) = make_uint2(0u, 0u);
+          *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out) + ooff) = make_uint2(0u, 0u);
         else
-          *reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(out) + eoff) = 0u;
+          *reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(out) + ooff) = 0u;
       } else {
-        float* o = static_cast<float*>(out) + eoff;
+        float* o = static_cast<float*>(out) + ooff;
 #pragma unroll
         for (int i = 0; i < kVec; ++i) o[i] = 0.f;
       }
@@ -100,13 +114,13 @@ __global__ void __launch_bounds__(kMergeThreads)
       }
     }
     if (kOutBf16) {
-      __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out) + eoff;
+      __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out) + ooff;
       if (kVec == 4)
         *reinterpret_cast<uint2*>(o) = make_uint2(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]));
       else
         *reinterpret_cast<uint32_t*>(o) = pack_bf16x2(acc[0], acc[1]);
     } else {
-      float* o = static_cast<float*>(out) + eoff;
+      float* o = static_cast<float*>(out) + ooff;
       if (kVec == 4)
         *reinterpret_cast<float4*>(o) = make_float4(acc[0], acc[1], acc[2], acc[3]);
       else

@@ -213,6 +213,25 @@ CP_API cp_status cp_ring_sim_static(const void* q, const void* k, const void* v,
                              int D, float scale, cp_dtype out_dtype, void* stream);
 
 /*
+ * cp_attn_merge_ulysses - cp_attn_merge of Ulysses head-shard partials, fused with the
+ * inverse exchange.
+ *
+ * Source: "Context parallelism", "Ulysses Attention" (the second all-to-all regroups the
+ * results by token) after the LSE merge of the ring blocks (as cp_attn_merge).  The merged
+ * rows are written straight to their sequence-sharded positions, so the head-sharded output
+ * is never stored and re-read; the result is bit-identical to cp_attn_merge followed by
+ * cp_ulysses_permute(direction 1).
+ * partials: fp32 [n_chunks][degree*B][S][H/degree][D] (attention on the head shards, shard p
+ *           = heads [p*H/degree, (p+1)*H/degree)); lses: fp32 [n_chunks][degree*B][H/degree][S].
+ * out:      out_dtype, sequence-sharded [degree][B][S/degree][H][D] (cp_ulysses_permute's
+ *           layout); out_lse: fp32 [B][H][S] (natural log), or NULL.
+ * Errors: S or H not divisible by degree -> CP_ERR_NOT_DIVISIBLE; otherwise as cp_attn_merge.
+ */
+CP_API cp_status cp_attn_merge_ulysses(const float* partials, const float* lses, int n_chunks, void* out,
+                                       float* out_lse, int degree, int B, int S, int H, int D, cp_dtype out_dtype,
+                                       void* stream);
+
+/*
  * cp_ulysses_anything_permute - the Ulysses exchange for shards of unequal size.
  *
  * Source: "Context parallelism", section "Ulysses Anything Attention": the sequence length

@@ -206,3 +206,35 @@ def test_bench_step_launch_configuration():
     o = o_seq.permute(1, 0, 2, 3, 4).reshape(B, S, H, D)
     lse = lse_h.view(P, B, H // P, S).permute(1, 0, 2, 3).reshape(B, H, S)  # head group p = heads 3p..3p+2
     assert_attn_close(o, lse, o_ref, lse_ref, "bench step (FLUX Ulysses-8 x ring-8)")
+
+
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32], ids=["bf16", "fp32"])
+@pytest.mark.parametrize("P,B,S,H,D,n", [(8, 1, 4608, 24, 128, 8), (4, 2, 200, 8, 64, 3), (3, 1, 99, 6, 128, 1)])
+def test_merge_ulysses_equals_merge_then_inverse_exchange(P, B, S, H, D, n, out_dtype):
+    g = torch.Generator().manual_seed(P * 7 + S)
+    parts = torch.randn(n, P * B, S, H // P, D, generator=g).cuda()
+    lses = (torch.randn(n, P * B, H // P, S, generator=g) * 3).cuda()
+    lses[0, 0, 0, :5] = -math.inf                    # an empty block for some rows
+    if n > 1:
+        lses[:, -1, -1, -1] = -math.inf              # a row with every block empty
+    o_h, l_h = binding.attn_merge(parts, lses, out_dtype=out_dtype)
+    want = binding.ulysses_permute(o_h.view(P, B, S, H // P, D), P, 1)
+    want_lse = l_h.view(P, B, H // P, S).permute(1, 0, 2, 3).reshape(B, H, S)
+    o, lse = binding.attn_merge_ulysses(parts, lses, P, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    assert torch.equal(o, want)
+    assert torch.equal(lse, want_lse)
+
+
+def test_bench_step_fused_merge_matches_oracle():
+    """The bench step with the merge fused into the inverse exchange, every element vs fp64."""
+    w, (q, k, v) = workload_inputs("flux_1024_ring8_ulysses8")
+    o_ref, lse_ref = workload_oracle("flux_1024_ring1")
+    P, B, S, H, D = 8, w.B, w.S, w.H, w.D
+    xs = [t.reshape(B, P, S // P, H, D).permute(1, 0, 2, 3, 4).contiguous().cuda() for t in (q, k, v)]
+    ys = binding.ulysses_permute_n(xs, P, 0)
+    view = lambda t: t.view(P * B, S, H // P, D)
+    parts, lses = binding.attn_fwd_blocks(view(ys[0]), view(ys[1]), view(ys[2]), even_bounds(S, 8), scale=w.scale)
+    o_seq, lse = binding.attn_merge_ulysses(parts, lses, P)
+    o = o_seq.permute(1, 0, 2, 3, 4).reshape(B, S, H, D)
+    assert_attn_close(o, lse, o_ref, lse_ref, "bench step, fused merge + inverse exchange")
