@@ -34,6 +34,15 @@ sys.path.insert(0, ROOT)
 WORKLOAD = "flux_1024_ring8_ulysses8"
 METRIC = "attention TFLOP/s (4*B*H*Sq*Skv*D) and % of B200 BF16 peak; merge/permute GB/s"
 UNIT = "TFLOP/s"
+STEP_WORKLOAD = ("FLUX.1-dev 1024x1024 joint attention B1 H24 S4608 D128: Ulysses-8 exchange of Q/K/V, "
+                 "ring-8 blockwise attention (8 x 576 keys) + LSE merge, inverse exchange of O")
+
+
+def step_config(world: int, B: int, S: int, H: int, D: int, P: int, n_blocks: int, l2: str) -> dict:
+    """The workload description shared by both arms of the bench (same keys, same workload)."""
+    return {"workload": STEP_WORKLOAD, "global_batch": world * B, "seq_len": S, "heads": H, "head_dim": D,
+            "ulysses_degree": P, "ring_degree": n_blocks,
+            "parallelism": f"replicas x{world} (single-GPU simulated degrees)", "l2": l2}
 
 # DRAM traffic of the timed attention launch (8 ring blocks, FLUX B1), from one ncu capture
 # of the same kernel on the B2 shape (profiles/attn_fwd_sm100__flux_b2_ring8.md):
@@ -384,14 +393,8 @@ def run_ours(args):
             "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) bf16, per-head RMS-normed Q/K; sha256 " + ",".join(
                 f"{k}:{v}" for k, v in sha.items()) + ")",
-            "config": {
-                "workload": ("FLUX.1-dev 1024x1024 joint attention B1 H24 S4608 D128: Ulysses-8 exchange of Q/K/V, "
-                             "ring-8 blockwise attention (8 x 576 keys) + LSE merge, inverse exchange of O"),
-                "global_batch": world * B, "seq_len": S, "heads": H, "head_dim": D,
-                "ulysses_degree": P, "ring_degree": n_blocks,
-                "parallelism": f"replicas x{world} (single-GPU simulated degrees)",
-                "l2": "flushed between timed steps (write of %d MiB > L2)" % (flush.numel() >> 20),
-            },
+            "config": step_config(world, B, S, H, D, P, n_blocks,
+                                  "flushed between timed steps (write of %d MiB > L2)" % (flush.numel() >> 20)),
             "roofline": {
                 "kernel": "attn_fwd_sm100 (8 ring blocks in one launch)",
                 "bound": "tensor",
@@ -513,10 +516,11 @@ def run_reference(args):
         "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-        "config": {"workload": "FLUX.1-dev 1024x1024 joint attention B1 H24 S4608 D128, ring-8 + LSE merge "
-                               f"(fp64 CPU oracle, {n_rows} sampled query rows per step)"},
+        "config": step_config(1, w.B, w.S, w.H, w.D, w.ulysses_degree, len(w.splits[0]),
+                              "host cores (fp64 oracle; no GPU cache involved)"),
         "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": _threads_used(), "kind": "oracle",
-                         "sample": f"{n_rows} of {w.S} query rows per step, all heads, 8 K/V blocks + merge"},
+                         "sample": f"{n_rows} of {w.S} query rows per step, all heads, 8 K/V blocks + merge "
+                                   "(the exchanges are index maps with no arithmetic: not timed)"},
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
