@@ -13,6 +13,8 @@
 #include <mutex>
 
 #include "../../include/cpattn.h"
+#include <nvtx3/nvToolsExt.h>
+
 #include "attn_fwd_sm100.cuh"
 #include "lse_merge.cuh"
 #include "ulysses_permute.cuh"
@@ -39,6 +41,15 @@ std::mutex g_mutex;
 DeviceInfo g_dev[kMaxDevices];
 int g_fault_next = 0;  // test hook consumed by the next attention launch
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+// An NVTX range around every public call, so that profilers show each call by name
+// (header-only NVTX3: without an attached tool the push and pop cost a few instructions).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -236,6 +247,7 @@ const char* cp_status_string(cp_status s) {
 
 cp_status cp_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H, int Sq,
                       int Skv, int D, float scale, cp_dtype out_dtype, void* stream) {
+  NvtxRange nvtx_range("cp_attn_fwd");
   cp_status st = check_attn_args(q, k, v, out, lse, B, H, Sq, Skv, D, scale, out_dtype);
   if (st != CP_OK || B == 0 || H == 0 || Sq == 0) return st;
   const int bounds[2] = {0, Skv};
@@ -245,6 +257,7 @@ cp_status cp_attn_fwd(const void* q, const void* k, const void* v, void* out, fl
 
 cp_status cp_attn_merge(const float* partials, const float* lses, int n_chunks, void* out, float* out_lse, int B,
                         int H, int Sq, int D, cp_dtype out_dtype, void* stream) {
+  NvtxRange nvtx_range("cp_attn_merge");
   if (B < 0 || H < 0 || Sq < 0) return CP_ERR_INVALID_ARG;
   if (n_chunks < 1 || n_chunks > CP_MAX_CHUNKS) return n_chunks < 1 ? CP_ERR_INVALID_ARG : CP_ERR_UNSUPPORTED;
   if (D != 64 && D != 128) return CP_ERR_UNSUPPORTED;
@@ -267,6 +280,7 @@ size_t cp_ring_sim_workspace_size(int n_chunks, int B, int H, int Sq, int D) {
 cp_status cp_attn_fwd_blocks(const void* q, const void* k, const void* v, const int* chunk_bounds, int n_chunks,
                              float* partials, float* lses, int B, int H, int Sq, int Skv, int D, float scale,
                              void* stream) {
+  NvtxRange nvtx_range("cp_attn_fwd_blocks");
   cp_status st = check_bounds(chunk_bounds, n_chunks, Skv);
   if (st != CP_OK) return st;
   st = check_attn_args(q, k, v, partials, lses, B, H, Sq, Skv, D, scale, CP_F32);
@@ -280,6 +294,7 @@ cp_status cp_attn_fwd_blocks(const void* q, const void* k, const void* v, const 
 cp_status cp_ring_sim(const void* q, const void* k, const void* v, const int* chunk_bounds, int n_chunks, void* out,
                       float* out_lse, int B, int H, int Sq, int Skv, int D, float scale, cp_dtype out_dtype,
                       void* workspace, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("cp_ring_sim");
   cp_status st = check_bounds(chunk_bounds, n_chunks, Skv);
   if (st != CP_OK) return st;
   st = check_attn_args(q, k, v, out, out_lse, B, H, Sq, Skv, D, scale, out_dtype);
@@ -331,6 +346,7 @@ extern "C" {
 cp_status cp_ring_sim_static(const void* q, const void* k, const void* v, const int* chunk_bounds, int n_chunks,
                              void* out, float* out_lse, int B, int H, int Sq, int Skv, int D, float scale,
                              cp_dtype out_dtype, void* stream) {
+  NvtxRange nvtx_range("cp_ring_sim_static");
   cp_status st = check_bounds(chunk_bounds, n_chunks, Skv);
   if (st != CP_OK) return st;
   st = check_attn_args(q, k, v, out, out_lse, B, H, Sq, Skv, D, scale, out_dtype);
@@ -358,6 +374,7 @@ size_t cp_usp_sim_workspace_size(int degree, int n_chunks, int B, int S, int H, 
 cp_status cp_usp_sim(const void* q, const void* k, const void* v, int degree, const int* chunk_bounds, int n_chunks,
                      void* out, float* out_lse, int B, int S, int H, int D, float scale, cp_dtype out_dtype,
                      void* workspace, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("cp_usp_sim");
   if (degree < 1 || B <= 0 || S <= 0 || H <= 0) return CP_ERR_INVALID_ARG;
   if (S % degree != 0 || H % degree != 0) return CP_ERR_NOT_DIVISIBLE;
   cp_status st = check_bounds(chunk_bounds, n_chunks, S);
@@ -404,6 +421,7 @@ cp_status cp_usp_sim(const void* q, const void* k, const void* v, int degree, co
 cp_status cp_ring_sim_fused(const void* q, const void* k, const void* v, const int* chunk_bounds, int n_chunks,
                             void* out, float* out_lse, int B, int H, int Sq, int Skv, int D, float scale,
                             cp_dtype out_dtype, void* stream) {
+  NvtxRange nvtx_range("cp_ring_sim_fused");
   cp_status st = check_bounds(chunk_bounds, n_chunks, Skv);
   if (st != CP_OK) return st;
   st = check_attn_args(q, k, v, out, out_lse, B, H, Sq, Skv, D, scale, out_dtype);
@@ -414,6 +432,7 @@ cp_status cp_ring_sim_fused(const void* q, const void* k, const void* v, const i
 
 cp_status cp_ulysses_permute_n(const void* const* srcs, void* const* dsts, int n_tensors, int degree, int B, int S,
                                int H, int D, int direction, int elem_bytes, void* stream) {
+  NvtxRange nvtx_range("cp_ulysses_permute_n");
   if (degree < 1 || B < 0 || S < 0 || H < 0 || D < 0) return CP_ERR_INVALID_ARG;
   if (direction != 0 && direction != 1) return CP_ERR_INVALID_ARG;
   if (elem_bytes != 2 && elem_bytes != 4) return CP_ERR_UNSUPPORTED;
@@ -469,6 +488,7 @@ cp_status cp_ulysses_permute_n(const void* const* srcs, void* const* dsts, int n
 
 cp_status cp_attn_merge_ulysses(const float* partials, const float* lses, int n_chunks, void* out, float* out_lse,
                                 int degree, int B, int S, int H, int D, cp_dtype out_dtype, void* stream) {
+  NvtxRange nvtx_range("cp_attn_merge_ulysses");
   if (degree < 1 || B < 0 || S < 0 || H < 0) return CP_ERR_INVALID_ARG;
   if (S % degree != 0 || H % degree != 0) return CP_ERR_NOT_DIVISIBLE;
   if (n_chunks < 1 || n_chunks > CP_MAX_CHUNKS) return n_chunks < 1 ? CP_ERR_INVALID_ARG : CP_ERR_UNSUPPORTED;
@@ -486,6 +506,7 @@ cp_status cp_attn_merge_ulysses(const float* partials, const float* lses, int n_
 cp_status cp_ulysses_anything_permute(const void* src, void* dst, int degree, const int* seq_bounds,
                                       const int* head_bounds, int B, int S, int H, int D, int direction, int elem_bytes,
                                       void* stream) {
+  NvtxRange nvtx_range("cp_ulysses_anything_permute");
   if (degree < 1 || B < 0 || S < 0 || H < 0 || D < 0 || !seq_bounds || !head_bounds) return CP_ERR_INVALID_ARG;
   if (degree > kPermuteMaxDegree) return CP_ERR_UNSUPPORTED;
   if (direction != 0 && direction != 1) return CP_ERR_INVALID_ARG;
@@ -539,6 +560,7 @@ cp_status cp_ulysses_anything_permute(const void* src, void* dst, int degree, co
 
 cp_status cp_ulysses_permute(const void* src, void* dst, int degree, int B, int S, int H, int D, int direction,
                              int elem_bytes, void* stream) {
+  NvtxRange nvtx_range("cp_ulysses_permute");
   // Pointers are checked by the batched form; nulls with empty sizes stay a no-op.
   if (degree < 1 || B < 0 || S < 0 || H < 0 || D < 0) return CP_ERR_INVALID_ARG;
   if (direction != 0 && direction != 1) return CP_ERR_INVALID_ARG;
