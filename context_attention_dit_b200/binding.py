@@ -18,7 +18,11 @@ from typing import Optional, Sequence
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libcpattn.so")
+# The debug build (libcpattn_debug.so, device-side bounds checks) is selected with
+# CPATTN_LIB=debug; any other value is taken as a path.
+_lib_env = os.environ.get("CPATTN_LIB", "")
+LIB_PATH = (os.path.join(_PKG, "libcpattn_debug.so") if _lib_env == "debug"
+            else _lib_env or os.path.join(_PKG, "libcpattn.so"))
 
 CP_OK = 0
 CP_ERR_INVALID_ARG = -1
@@ -27,6 +31,7 @@ CP_ERR_NOT_DIVISIBLE = -3
 CP_ERR_MISALIGNED = -4
 CP_ERR_CUDA = -5
 CP_ERR_TIMEOUT = -6
+CP_ERR_BOUNDS = -7
 CP_BF16 = 0
 CP_F32 = 1
 CP_MAX_CHUNKS = 64

@@ -16,6 +16,9 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libcpattn.so")
+# Debug build: every global index a kernel computes is checked against its buffer
+# (-DCP_DEBUG); a violation is reported as CP_ERR_BOUNDS instead of touching memory.
+LIB_DEBUG = os.path.join(PKG, "libcpattn_debug.so")
 
 
 def nvcc_path() -> str:
@@ -60,6 +63,16 @@ def build(force: bool = False, verbose: bool = False, extra=(), out: str | None 
     return out
 
 
+def build_debug(force: bool = False) -> str:
+    """Compile the bounds-checking debug library (libcpattn_debug.so)."""
+    if not force and os.path.exists(LIB_DEBUG) and all(
+            os.path.getmtime(s) <= os.path.getmtime(LIB_DEBUG) for s in sources() + [__file__]):
+        return LIB_DEBUG
+    return build(extra=("-DCP_DEBUG",), out=LIB_DEBUG)
+
+
 if __name__ == "__main__":
     build(force=True, verbose="-v" in sys.argv)
     print(LIB)
+    if "--debug" in sys.argv:
+        print(build_debug(force=True))

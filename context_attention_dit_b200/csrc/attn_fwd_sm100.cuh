@@ -95,6 +95,7 @@ struct AttnParams {
   long long out_chunk_stride;
   float* lse;                // block c at lse + c*lse_chunk_stride, [B][H][Sq]; may be null
   long long lse_chunk_stride;
+  long long out_elems, lse_elems;  // extents of out and lse (checked in debug builds)
   int* status;               // device status word
   int fuse;                  // 1: one running softmax over all blocks, one merged output
   int fault;                 // test hook: 1 = the producer never loads the CTA's first K tile
@@ -575,16 +576,17 @@ template <int D>
 __device__ __forceinline__ void write_empty_row(const AttnParams& p, int c, const UnitCoord& uc, int s_row) {
   const size_t o_off = static_cast<size_t>(c) * p.out_chunk_stride +
                        ((static_cast<size_t>(uc.b) * p.Sq + s_row) * p.H + uc.h) * D;
-  if (p.out_f32) {
-    float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out) + o_off);
-    for (int i = 0; i < D / 4; ++i) o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-  } else {
-    uint4* o = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + o_off);
-    for (int i = 0; i < D / 8; ++i) o[i] = make_uint4(0u, 0u, 0u, 0u);
+  if (in_bounds(static_cast<long long>(o_off), D, p.out_elems)) {
+    if (p.out_f32) {
+      float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out) + o_off);
+      for (int i = 0; i < D / 4; ++i) o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    } else {
+      uint4* o = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + o_off);
+      for (int i = 0; i < D / 8; ++i) o[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
   }
-  if (p.lse)
-    p.lse[static_cast<size_t>(c) * p.lse_chunk_stride + (static_cast<size_t>(uc.b) * p.H + uc.h) * p.Sq + s_row] =
-        -INFINITY;
+  const size_t li = static_cast<size_t>(c) * p.lse_chunk_stride + (static_cast<size_t>(uc.b) * p.H + uc.h) * p.Sq + s_row;
+  if (p.lse && in_bounds(static_cast<long long>(li), 1, p.lse_elems)) p.lse[li] = -INFINITY;
 }
 
 // Softmax warpgroup k (key half k): every tile of every block of every unit; at a
@@ -724,13 +726,14 @@ __device__ __forceinline__ void attn_epilogue(const AttnParams& p, uint8_t* smem
 #pragma unroll
         for (int i = 0; i < D; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * c0f);
       }
-      if (row_ok) {
+      if (row_ok && in_bounds(static_cast<long long>(o_off), D, p.out_elems)) {
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) store_row<D>(p, o_off, *reinterpret_cast<const uint32_t(*)[32]>(r + cc * 32), cc);
       }
-      if (row_ok && p.lse)
-        p.lse[static_cast<size_t>(c) * p.lse_chunk_stride + (static_cast<size_t>(uc.b) * p.H + uc.h) * p.Sq +
-              s_row] = (mx + log2f(lsum)) * 0.69314718055994530942f;
+      const size_t li =
+          static_cast<size_t>(c) * p.lse_chunk_stride + (static_cast<size_t>(uc.b) * p.H + uc.h) * p.Sq + s_row;
+      if (row_ok && p.lse && in_bounds(static_cast<long long>(li), 1, p.lse_elems))
+        p.lse[li] = (mx + log2f(lsum)) * 0.69314718055994530942f;
       ++nch;
     }
   }

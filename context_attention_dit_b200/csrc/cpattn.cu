@@ -22,9 +22,7 @@
 using namespace cpattn;
 
 static_assert(kMaxChunks == CP_MAX_CHUNKS, "chunk limit mismatch");
-
-// Device status word: kernels record CP_ERR_TIMEOUT here when a bounded wait runs out.
-__device__ int g_cp_status = 0;
+static_assert(kDevTimeout == CP_ERR_TIMEOUT && kDevBounds == CP_ERR_BOUNDS, "device status codes mismatch");
 
 namespace {
 
@@ -136,6 +134,12 @@ cp_status launch_attn(const void* q, const void* k, const void* v, const int* bo
   p.out_chunk_stride = out_chunk_stride;
   p.lse = lse;
   p.lse_chunk_stride = lse_chunk_stride;
+  {  // output extents: one [B][Sq][H][D] output (and [B][H][Sq] LSE) per written block
+    const long long one_o = static_cast<long long>(B) * Sq * H * D, one_l = static_cast<long long>(B) * H * Sq;
+    const int n_out = (fuse || out_chunk_stride == 0) ? 1 : n_chunks;
+    p.out_elems = out_chunk_stride ? out_chunk_stride * (n_out - 1) + one_o : one_o;
+    p.lse_elems = lse_chunk_stride ? lse_chunk_stride * (n_out - 1) + one_l : one_l;
+  }
   p.status = dev->status;
   for (int i = 0; i <= n_chunks; ++i) p.bounds[i] = bounds[i];
   p.fuse = fuse;
@@ -241,6 +245,7 @@ const char* cp_status_string(cp_status s) {
     case CP_ERR_MISALIGNED: return "CP_ERR_MISALIGNED: device pointer not 16-byte aligned";
     case CP_ERR_CUDA: return "CP_ERR_CUDA: CUDA runtime or driver error";
     case CP_ERR_TIMEOUT: return "CP_ERR_TIMEOUT: a device-side wait ran out";
+    case CP_ERR_BOUNDS: return "CP_ERR_BOUNDS: a debug build caught an index outside its buffer";
   }
   return "unknown cp_status";
 }

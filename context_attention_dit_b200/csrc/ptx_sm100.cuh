@@ -11,6 +11,25 @@ namespace cpattn {
 // Status codes written to the device status word (mirror cp_status in cpattn.h).
 constexpr int kDevOk = 0;
 constexpr int kDevTimeout = -6;
+constexpr int kDevBounds = -7;
+
+// Device status word: kernels record kDevTimeout here when a bounded wait runs out, and
+// debug builds record kDevBounds when a computed index falls outside its buffer.
+__device__ int g_cp_status = 0;
+
+// Debug builds (-DCP_DEBUG) check every global index a kernel computes (TMA accesses are
+// bounded by the hardware) against the extent of its buffer: a violation records
+// kDevBounds and returns false, so that the caller skips the access instead of faulting.
+// Release builds compile the check away.
+__device__ __forceinline__ bool in_bounds(long long first, long long count, long long extent) {
+#ifdef CP_DEBUG
+  if (first < 0 || count < 0 || first + count > extent) {
+    atomicExch(&g_cp_status, kDevBounds);
+    return false;
+  }
+#endif
+  return true;
+}
 
 // A bounded wait gives up after this many SM clock cycles (~1 s at 1.9 GHz).
 constexpr long long kWaitLimitCycles = 2000000000LL;

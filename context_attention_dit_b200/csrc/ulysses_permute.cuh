@@ -17,6 +17,8 @@
 
 #include <cstdint>
 
+#include "ptx_sm100.cuh"
+
 namespace cpattn {
 
 constexpr int kPermuteThreads = 128;
@@ -48,23 +50,20 @@ __global__ void __launch_bounds__(kPermuteThreads)
   const long long S = static_cast<long long>(Sp) * P;
   const long long x0 = static_cast<long long>(pb) * Sp * row_vecs + i;                     // X row stride row_vecs
   const long long y0 = ((static_cast<long long>(q) * B + b) * S + static_cast<long long>(p) * Sp) * piece_vecs + w;
+  const long long total = static_cast<long long>(P) * B * Sp * row_vecs;  // vectors per tensor
   for (int s0 = blockIdx.y * kPermuteRows; s0 < Sp; s0 += gridDim.y * kPermuteRows) {
     V v[kPermuteRows];
 #pragma unroll
     for (int r = 0; r < kPermuteRows; ++r) {
       const int sl = s0 + r;
-      if (sl < Sp) v[r] = direction == 0 ? src[x0 + static_cast<long long>(sl) * row_vecs]
-                                         : src[y0 + static_cast<long long>(sl) * piece_vecs];
+      const long long xi = x0 + static_cast<long long>(sl) * row_vecs, yi = y0 + static_cast<long long>(sl) * piece_vecs;
+      if (sl < Sp && in_bounds(direction == 0 ? xi : yi, 1, total)) v[r] = src[direction == 0 ? xi : yi];
     }
 #pragma unroll
     for (int r = 0; r < kPermuteRows; ++r) {
       const int sl = s0 + r;
-      if (sl < Sp) {
-        if (direction == 0)
-          dst[y0 + static_cast<long long>(sl) * piece_vecs] = v[r];
-        else
-          dst[x0 + static_cast<long long>(sl) * row_vecs] = v[r];
-      }
+      const long long xi = x0 + static_cast<long long>(sl) * row_vecs, yi = y0 + static_cast<long long>(sl) * piece_vecs;
+      if (sl < Sp && in_bounds(direction == 0 ? yi : xi, 1, total)) dst[direction == 0 ? yi : xi] = v[r];
     }
   }
 }
@@ -108,22 +107,20 @@ __global__ void __launch_bounds__(kPermuteThreads)
   const long long xs = static_cast<long long>(H) * D / VE;
   const long long y0 = (static_cast<long long>(B) * S * hq * D + (static_cast<long long>(b) * S + s0) * Hq * D + w) / VE;
   const long long ys = Hq * D / VE;
+  const long long total = static_cast<long long>(B) * S * H * D / VE;  // vectors per buffer
   for (int sl0 = blockIdx.y * kPermuteRows; sl0 < Sp; sl0 += gridDim.y * kPermuteRows) {
     V v[kPermuteRows];
 #pragma unroll
     for (int r = 0; r < kPermuteRows; ++r) {
       const int sl = sl0 + r;
-      if (sl < Sp) v[r] = direction == 0 ? src[x0 + sl * xs] : src[y0 + sl * ys];
+      const long long si = direction == 0 ? x0 + sl * xs : y0 + sl * ys;
+      if (sl < Sp && in_bounds(si, 1, total)) v[r] = src[si];
     }
 #pragma unroll
     for (int r = 0; r < kPermuteRows; ++r) {
       const int sl = sl0 + r;
-      if (sl < Sp) {
-        if (direction == 0)
-          dst[y0 + sl * ys] = v[r];
-        else
-          dst[x0 + sl * xs] = v[r];
-      }
+      const long long di = direction == 0 ? y0 + sl * ys : x0 + sl * xs;
+      if (sl < Sp && in_bounds(di, 1, total)) dst[di] = v[r];
     }
   }
 }
@@ -138,7 +135,11 @@ __global__ void __launch_bounds__(256) lse_regroup_kernel(const float* __restric
   const int b = pb - p * B;
   const float* s = src + static_cast<long long>(pb) * block;
   float* d = dst + (static_cast<long long>(b) * P + p) * block;
-  for (long long i = blockIdx.x * 256LL + threadIdx.x; i < block; i += gridDim.x * 256LL) d[i] = s[i];
+  const long long total = static_cast<long long>(P) * B * block;
+  for (long long i = blockIdx.x * 256LL + threadIdx.x; i < block; i += gridDim.x * 256LL)
+    if (in_bounds(static_cast<long long>(pb) * block + i, 1, total) &&
+        in_bounds((static_cast<long long>(b) * P + p) * block + i, 1, total))
+      d[i] = s[i];
 }
 
 }  // namespace cpattn

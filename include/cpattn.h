@@ -54,7 +54,9 @@ typedef enum {
   CP_ERR_NOT_DIVISIBLE = -3, /* S or H not divisible by the Ulysses degree; uneven split without "anything" */
   CP_ERR_MISALIGNED = -4,    /* a device pointer not 16-byte aligned (TMA and vector access need it) */
   CP_ERR_CUDA = -5,          /* a CUDA runtime/driver call failed (no device, launch failure, ...) */
-  CP_ERR_TIMEOUT = -6        /* a device-side bounded wait ran out; the kernel stopped and returned */
+  CP_ERR_TIMEOUT = -6,       /* a device-side bounded wait ran out; the kernel stopped and returned */
+  CP_ERR_BOUNDS = -7         /* debug builds (-DCP_DEBUG): a kernel computed an index outside its
+                                buffer and skipped that access */
 } cp_status;
 
 typedef enum { CP_BF16 = 0, CP_F32 = 1 } cp_dtype;

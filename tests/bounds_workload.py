@@ -1,0 +1,64 @@
+"""A deterministic set of calls touching every kernel path (ragged shapes, empty blocks and
+shards, both output types), used by tests/test_debug_bounds_gpu.py to run the same work
+through the release and the bounds-checking debug library.  Prints one JSON object:
+call name -> SHA-256 of its outputs, plus the device status after every call."""
+
+import hashlib
+import json
+import sys
+
+import torch
+
+from context_attention_dit_b200 import binding
+from context_attention_dit_b200.inputs import make_qkv
+
+
+def _digest(*ts):
+    h = hashlib.sha256()
+    for t in ts:
+        h.update(t.detach().contiguous().view(torch.uint8).cpu().numpy().tobytes())
+    return h.hexdigest()[:24]
+
+
+def run():
+    torch.cuda.set_device(0)
+    out = {}
+
+    def record(name, *ts):
+        torch.cuda.synchronize()
+        out[name] = {"status": binding.last_device_status(), "digest": _digest(*ts)}
+
+    for B, H, Sq, Skv, D, dt in ((1, 2, 1, 1, 128, torch.bfloat16), (2, 3, 129, 300, 128, torch.float32),
+                                 (1, 2, 300, 77, 64, torch.bfloat16), (1, 4, 1391, 1391, 128, torch.bfloat16)):
+        q, k, v = (t.cuda() for t in make_qkv(B, H, Sq, Skv, D, seed=3))
+        record(f"attn_{B}x{H}x{Sq}x{Skv}x{D}", *binding.attn_fwd(q, k, v, out_dtype=dt))
+    q, k, v = (t.cuda() for t in make_qkv(1, 2, 450, 450, 128, seed=4))
+    for bounds in ([0, 0, 130, 130, 450], [0, 5, 6, 450], [0, 450, 450]):
+        o, lse, _ = binding.ring_sim(q, k, v, bounds)
+        record(f"ring_{bounds}", o, lse)
+        record(f"ring_fused_{bounds}", *binding.ring_sim_fused(q, k, v, bounds, out_dtype=torch.float32))
+    P, B, S, H, D = 4, 2, 384, 8, 128
+    x = [t.cuda() for t in make_qkv(P * B, H // P, S, S, D, seed=5)]
+    parts, lses = binding.attn_fwd_blocks(*x, [0, 100, 101, 384])
+    record("blocks", parts, lses)
+    record("merge", *binding.attn_merge(parts, lses))
+    record("merge_ulysses", *binding.attn_merge_ulysses(parts, lses, P))
+    src = torch.randn(P, B, S // P, H, D, generator=torch.Generator().manual_seed(6)).bfloat16().cuda()
+    y = binding.ulysses_permute(src, P, 0)
+    record("permute", y, binding.ulysses_permute(y, P, 1))
+    record("permute_n", *binding.ulysses_permute_n([src, src.clone()], P, 0))
+    for Pa, Sa, Ha, Da, sb, hb in ((4, 10, 3, 64, [0, 3, 6, 8, 10], [0, 1, 2, 3, 3]),
+                                   (3, 9, 6, 5, [0, 0, 4, 9], [0, 2, 4, 6])):
+        xa = torch.randn(2 * Sa * Ha * Da, generator=torch.Generator().manual_seed(7)).bfloat16().cuda()
+        ya = binding.ulysses_anything_permute(xa, Pa, sb, hb, 2, Sa, Ha, Da, 0)
+        record(f"anything_{Pa}_{Sa}_{Ha}_{Da}", ya, binding.ulysses_anything_permute(ya, Pa, sb, hb, 2, Sa, Ha, Da, 1))
+    shards = [t.reshape(1, 2, 128, 4, 128).permute(1, 0, 2, 3, 4).contiguous().cuda()
+              for t in make_qkv(1, 4, 256, 256, 128, seed=8)]
+    o, lse, _ = binding.usp_sim(*shards, 2, [0, 100, 256])
+    record("usp", o, lse)
+    return out
+
+
+if __name__ == "__main__":
+    print(json.dumps(run()))
+    sys.stdout.flush()

@@ -49,7 +49,7 @@ def test_sources_compile_and_export_header(tmp_path):
 
 def test_version_and_strings(lib):
     assert lib.cp_version() == 100
-    for code in (0, -1, -2, -3, -4, -5, -6):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7):
         assert binding.status_string(code).startswith("CP_")
 
 
