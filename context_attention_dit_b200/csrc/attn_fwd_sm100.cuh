@@ -585,8 +585,14 @@ __device__ __forceinline__ void write_empty_row(const AttnParams& p, int c, cons
       for (int i = 0; i < D / 8; ++i) o[i] = make_uint4(0u, 0u, 0u, 0u);
     }
   }
+#ifdef CP_DEBUG
   const size_t li = static_cast<size_t>(c) * p.lse_chunk_stride + (static_cast<size_t>(uc.b) * p.H + uc.h) * p.Sq + s_row;
   if (p.lse && in_bounds(static_cast<long long>(li), 1, p.lse_elems)) p.lse[li] = -INFINITY;
+#else
+  if (p.lse)
+    p.lse[static_cast<size_t>(c) * p.lse_chunk_stride + (static_cast<size_t>(uc.b) * p.H + uc.h) * p.Sq + s_row] =
+        -INFINITY;
+#endif
 }
 
 // Softmax warpgroup k (key half k): every tile of every block of every unit; at a
@@ -730,10 +736,16 @@ __device__ __forceinline__ void attn_epilogue(const AttnParams& p, uint8_t* smem
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) store_row<D>(p, o_off, *reinterpret_cast<const uint32_t(*)[32]>(r + cc * 32), cc);
       }
+#ifdef CP_DEBUG
       const size_t li =
           static_cast<size_t>(c) * p.lse_chunk_stride + (static_cast<size_t>(uc.b) * p.H + uc.h) * p.Sq + s_row;
       if (row_ok && p.lse && in_bounds(static_cast<long long>(li), 1, p.lse_elems))
         p.lse[li] = (mx + log2f(lsum)) * 0.69314718055994530942f;
+#else
+      if (row_ok && p.lse)
+        p.lse[static_cast<size_t>(c) * p.lse_chunk_stride + (static_cast<size_t>(uc.b) * p.H + uc.h) * p.Sq +
+              s_row] = (mx + log2f(lsum)) * 0.69314718055994530942f;
+#endif
       ++nch;
     }
   }

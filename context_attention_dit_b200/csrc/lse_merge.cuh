@@ -46,13 +46,15 @@ __global__ void __launch_bounds__(kMergeThreads)
     const int h = rem / ST;
     const int st = rem - h * ST;
     const int s = s0 + st;
+#ifdef CP_DEBUG
     const long long li = c * lse_stride + (static_cast<long long>(b) * H + h) * Sq + s;
     lse_s[idx] = s < Sq && in_bounds(li, 1, n * lse_stride) ? __ldg(lses + li) : -INFINITY;
+#else
+    lse_s[idx] = s < Sq ? __ldg(lses + c * lse_stride + (static_cast<long long>(b) * H + h) * Sq + s) : -INFINITY;
+#endif
   }
   __syncthreads();
   const int lane = threadIdx.x & 31;
-  const long long rows_total = lse_stride;  // B*H*Sq rows in every block and in the output
-  (void)rows_total;
   for (int r = threadIdx.x >> 5; r < HS; r += kMergeThreads / 32) {
     const int st = r / H;
     const int h = r - st * H;
@@ -78,6 +80,7 @@ __global__ void __launch_bounds__(kMergeThreads)
 #ifdef CP_DEBUG
     // The row's partial vectors (every block), its output vector and its LSE.  The whole
     // warp skips the row, so that the shuffles below stay converged.
+    const long long rows_total = lse_stride;  // B*H*Sq rows in every block and in the output
     const bool ok = in_bounds(eoff + (n - 1) * part_stride, kVec, n * part_stride) &&
                     in_bounds(ooff, kVec, rows_total * D) && in_bounds(lrow, 1, rows_total);
     if (!__all_sync(0xffffffffu, ok)) continue;
