@@ -46,12 +46,12 @@ def step_config(world: int, B: int, S: int, H: int, D: int, P: int, n_blocks: in
 
 # DRAM traffic of the timed attention launch (8 ring blocks, FLUX B1), from one ncu capture
 # of the same kernel on the B2 shape (profiles/attn_fwd_sm100__flux_b2_ring8.md):
-# dram__bytes_read.sum + dram__bytes_write.sum = 185.73 + 862.05 MB, halved to one B1 launch
+# dram__bytes_read.sum + dram__bytes_write.sum = 186.38 + 860.91 MB, halved to one B1 launch
 # (the B1 launch processes half the units; Q/K/V reads and partial writes scale with them).
 # It describes only the kernel source it was captured on, identified by its SHA-256.
 ATTN_TRAFFIC = {
-    "kernel_sha256": "865bd87726044ea2ec385acff9c4d10946c62fe02430734494319448dadfcea7",
-    "bytes_per_launch": (185_726_976 + 862_048_000) // 2,
+    "kernel_sha256": "7f9867163754f9086e8eed92df542cb8c6d4fe4094ee51cb2303033950e6006a",
+    "bytes_per_launch": (186_379_776 + 860_907_008) // 2,
 }
 
 
