@@ -40,8 +40,11 @@ EXPORTS = (
     "cp_attn_fwd", "cp_attn_fwd_blocks", "cp_attn_merge", "cp_ring_sim_workspace_size", "cp_ring_sim",
     "cp_ring_sim_fused", "cp_ring_sim_static", "cp_ulysses_permute", "cp_ulysses_permute_n", "cp_ring_bounds",
     "cp_debug_set_fault", "cp_last_device_status", "cp_status_string", "cp_version", "cp_usp_sim_workspace_size",
-    "cp_usp_sim", "cp_ulysses_anything_permute", "cp_attn_merge_ulysses",
+    "cp_usp_sim", "cp_ulysses_anything_permute", "cp_attn_merge_ulysses", "cp_peer_alloc", "cp_peer_open",
+    "cp_peer_close", "cp_peer_free", "cp_ulysses_push_n", "cp_peer_barrier", "cp_ring_fetch_block",
 )
+CP_PEER_MAX = 16
+CP_IPC_HANDLE_BYTES = 64
 
 _lib = None
 
@@ -80,6 +83,13 @@ def load() -> ctypes.CDLL:
     lib.cp_ulysses_permute_n.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), i, i, i, i, i, i, i, i, vp]
     lib.cp_ulysses_permute_n.restype = ctypes.c_int
     lib.cp_ring_bounds.argtypes = [i, i, i, ip]
+    lib.cp_peer_alloc.argtypes = [sz, ctypes.POINTER(vp), ctypes.c_char_p]
+    lib.cp_peer_open.argtypes = [ctypes.c_char_p, ctypes.POINTER(vp)]
+    lib.cp_peer_close.argtypes = [vp]
+    lib.cp_peer_free.argtypes = [vp]
+    lib.cp_ulysses_push_n.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), i, i, i, i, i, i, i, i, i, vp]
+    lib.cp_peer_barrier.argtypes = [ctypes.POINTER(vp), i, i, ctypes.c_uint, vp]
+    lib.cp_ring_fetch_block.argtypes = [vp, vp, i, i, i, i, i, i, i, i, i, vp]
     lib.cp_debug_set_fault.argtypes = [i]
     lib.cp_debug_set_fault.restype = ctypes.c_int
     lib.cp_last_device_status.argtypes = [vp]
@@ -87,7 +97,8 @@ def load() -> ctypes.CDLL:
     lib.cp_status_string.restype = ctypes.c_char_p
     lib.cp_version.argtypes = []
     for name in ("cp_attn_fwd", "cp_attn_fwd_blocks", "cp_attn_merge", "cp_ring_sim", "cp_ring_sim_static", "cp_ulysses_permute",
-                 "cp_ring_bounds", "cp_last_device_status"):
+                 "cp_ring_bounds", "cp_last_device_status", "cp_peer_alloc", "cp_peer_open", "cp_peer_close",
+                 "cp_peer_free", "cp_ulysses_push_n", "cp_peer_barrier", "cp_ring_fetch_block"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -458,3 +469,76 @@ def debug_set_fault(mode: int):
 def last_device_status(stream=None) -> int:
     s = torch.cuda.current_stream() if stream is None else stream
     return int(load().cp_last_device_status(ctypes.c_void_p(s.cuda_stream)))
+
+
+# ------------------------------------------------------------------ one process per GPU
+# Raw device pointers (ints) in and out: peer buffers are not torch allocations.
+
+
+def peer_alloc(nbytes: int):
+    """A zero-filled device buffer other processes can map; returns ``(ptr, handle bytes)``."""
+    ptr = ctypes.c_void_p()
+    handle = ctypes.create_string_buffer(CP_IPC_HANDLE_BYTES)
+    _check(load().cp_peer_alloc(int(nbytes), ctypes.byref(ptr), handle), "cp_peer_alloc")
+    return int(ptr.value), handle.raw
+
+
+def peer_open(handle: bytes) -> int:
+    """Map another process's :func:`peer_alloc` buffer; returns the device pointer."""
+    if len(handle) != CP_IPC_HANDLE_BYTES:
+        raise ValueError(f"an IPC handle has {CP_IPC_HANDLE_BYTES} bytes, got {len(handle)}")
+    ptr = ctypes.c_void_p()
+    _check(load().cp_peer_open(ctypes.create_string_buffer(bytes(handle), CP_IPC_HANDLE_BYTES), ctypes.byref(ptr)),
+           "cp_peer_open")
+    return int(ptr.value)
+
+
+def peer_close(ptr: int):
+    _check(load().cp_peer_close(ctypes.c_void_p(ptr)), "cp_peer_close")
+
+
+def peer_free(ptr: int):
+    _check(load().cp_peer_free(ctypes.c_void_p(ptr)), "cp_peer_free")
+
+
+def ulysses_push_n(srcs: Sequence[int], dsts: Sequence[Sequence[int]], rank: int, degree: int, B: int, S: int, H: int,
+                   D: int, direction: int, elem_bytes: int, stream: int):
+    """This rank's half of a Ulysses all-to-all (see cp_ulysses_push_n): ``dsts[t][q]`` is
+    tensor t's buffer on rank q."""
+    n = len(srcs)
+    if n < 1 or len(dsts) != n or any(len(row) != degree for row in dsts):
+        raise ValueError("dsts needs one row of degree pointers per source")
+    sp = (ctypes.c_void_p * n)(*[int(x) for x in srcs])
+    dp = (ctypes.c_void_p * (n * degree))(*[int(x) for row in dsts for x in row])
+    _check(load().cp_ulysses_push_n(sp, dp, n, rank, degree, B, S, H, D, direction, elem_bytes, ctypes.c_void_p(stream)),
+           "cp_ulysses_push_n")
+
+
+def peer_barrier(pads: Sequence[int], rank: int, epoch: int, stream: int):
+    """Signal every rank's pad and wait (bounded) for every rank's signal (see cp_peer_barrier)."""
+    n = len(pads)
+    pp = (ctypes.c_void_p * n)(*[int(x) for x in pads])
+    _check(load().cp_peer_barrier(pp, rank, n, ctypes.c_uint(epoch & 0xFFFFFFFF), ctypes.c_void_p(stream)),
+           "cp_peer_barrier")
+
+
+def ring_fetch_block(dst: int, src: int, B: int, rows: int, H: int, D: int, dst_S: int, dst_row0: int, src_S: int,
+                     src_row0: int, elem_bytes: int, stream: int):
+    """Copy-engine copy of rows of a ``[B][S][H][D]`` tensor (see cp_ring_fetch_block)."""
+    _check(load().cp_ring_fetch_block(ctypes.c_void_p(dst), ctypes.c_void_p(src), B, rows, H, D, dst_S, dst_row0,
+                                      src_S, src_row0, elem_bytes, ctypes.c_void_p(stream)), "cp_ring_fetch_block")
+
+
+class _DeviceMemory:
+    """A raw device range seen by torch through the CUDA array interface (no copy)."""
+
+    def __init__(self, ptr: int, nbytes: int):
+        self.__cuda_array_interface__ = {"shape": (int(nbytes),), "typestr": "|u1", "data": (int(ptr), False),
+                                         "version": 3, "strides": None, "stream": None}
+
+
+def device_tensor(ptr: int, shape, dtype, device) -> torch.Tensor:
+    """A contiguous torch tensor over ``ptr`` (memory owned elsewhere; no copy)."""
+    nbytes = int(torch.Size(shape).numel()) * torch.empty((), dtype=dtype).element_size()
+    raw = torch.as_tensor(_DeviceMemory(ptr, max(nbytes, 1)), device=device)
+    return raw[:nbytes].view(dtype).view(shape)

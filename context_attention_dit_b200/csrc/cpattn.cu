@@ -17,12 +17,15 @@
 
 #include "attn_fwd_sm100.cuh"
 #include "lse_merge.cuh"
+#include "peer.cuh"
 #include "ulysses_permute.cuh"
 
 using namespace cpattn;
 
 static_assert(kMaxChunks == CP_MAX_CHUNKS, "chunk limit mismatch");
 static_assert(kDevTimeout == CP_ERR_TIMEOUT && kDevBounds == CP_ERR_BOUNDS, "device status codes mismatch");
+static_assert(kPeerMax == CP_PEER_MAX, "peer limit mismatch");
+static_assert(sizeof(cudaIpcMemHandle_t) == CP_IPC_HANDLE_BYTES, "IPC handle size mismatch");
 
 namespace {
 
@@ -50,6 +53,8 @@ struct NvtxRange {
 };
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// LSE arrays are read and written one float at a time.
+inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 cp_status device_info(DeviceInfo** out) {
   int dev = 0;
@@ -100,7 +105,7 @@ cp_status check_attn_args(const void* q, const void* k, const void* v, const voi
   if (!q || !out) return CP_ERR_INVALID_ARG;
   if (Skv > 0 && (!k || !v)) return CP_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(out) || (Skv > 0 && (!aligned16(k) || !aligned16(v))) ||
-      (lse && !aligned16(lse)))
+      (lse && !aligned4(lse)))
     return CP_ERR_MISALIGNED;
   // 32-bit limits: TMA coordinates, unit counts.
   const long long n_qt = (Sq + kBM - 1) / kBM;
@@ -234,7 +239,7 @@ inline size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255);
 
 extern "C" {
 
-int cp_version(void) { return 100; }
+int cp_version(void) { return 101; }
 
 const char* cp_status_string(cp_status s) {
   switch (s) {
@@ -269,7 +274,7 @@ cp_status cp_attn_merge(const float* partials, const float* lses, int n_chunks, 
   if (out_dtype != CP_BF16 && out_dtype != CP_F32) return CP_ERR_INVALID_ARG;
   if (B == 0 || H == 0 || Sq == 0) return CP_OK;
   if (!partials || !lses || !out) return CP_ERR_INVALID_ARG;
-  if (!aligned16(partials) || !aligned16(lses) || !aligned16(out) || (out_lse && !aligned16(out_lse)))
+  if (!aligned16(partials) || !aligned4(lses) || !aligned16(out) || (out_lse && !aligned4(out_lse)))
     return CP_ERR_MISALIGNED;
   return launch_merge(partials, lses, n_chunks, out, out_lse, B, H, Sq, D, out_dtype,
                       static_cast<cudaStream_t>(stream));
@@ -501,7 +506,7 @@ cp_status cp_attn_merge_ulysses(const float* partials, const float* lses, int n_
   if (out_dtype != CP_BF16 && out_dtype != CP_F32) return CP_ERR_INVALID_ARG;
   if (B == 0 || H == 0 || S == 0) return CP_OK;
   if (!partials || !lses || !out) return CP_ERR_INVALID_ARG;
-  if (!aligned16(partials) || !aligned16(lses) || !aligned16(out) || (out_lse && !aligned16(out_lse)))
+  if (!aligned16(partials) || !aligned4(lses) || !aligned16(out) || (out_lse && !aligned4(out_lse)))
     return CP_ERR_MISALIGNED;
   if (static_cast<long long>(degree) * B > 65535) return CP_ERR_UNSUPPORTED;
   return launch_merge(partials, lses, n_chunks, out, out_lse, degree * B, H / degree, S, D, out_dtype,
@@ -601,6 +606,151 @@ cp_status cp_last_device_status(void* stream) {
     if (cudaMemcpyToSymbol(g_cp_status, &zero, sizeof(int)) != cudaSuccess) return CP_ERR_CUDA;
   }
   return static_cast<cp_status>(v);
+}
+
+// ------------------------------------------------------------------ one process per GPU
+
+cp_status cp_peer_alloc(size_t bytes, void** dptr, void* handle) {
+  NvtxRange nvtx_range("cp_peer_alloc");
+  if (bytes == 0 || !dptr || !handle) return CP_ERR_INVALID_ARG;
+  *dptr = nullptr;
+  void* p = nullptr;
+  if (cudaMalloc(&p, bytes) != cudaSuccess) return CP_ERR_CUDA;
+  cudaIpcMemHandle_t h;
+  if (cudaMemset(p, 0, bytes) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess ||
+      cudaIpcGetMemHandle(&h, p) != cudaSuccess) {
+    cudaFree(p);
+    return CP_ERR_CUDA;
+  }
+  std::memcpy(handle, &h, sizeof(h));
+  *dptr = p;
+  return CP_OK;
+}
+
+cp_status cp_peer_open(const void* handle, void** dptr) {
+  NvtxRange nvtx_range("cp_peer_open");
+  if (!handle || !dptr) return CP_ERR_INVALID_ARG;
+  *dptr = nullptr;
+  cudaIpcMemHandle_t h;
+  std::memcpy(&h, handle, sizeof(h));
+  void* p = nullptr;
+  if (cudaIpcOpenMemHandle(&p, h, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess) return CP_ERR_CUDA;
+  *dptr = p;
+  return CP_OK;
+}
+
+cp_status cp_peer_close(void* dptr) {
+  if (!dptr) return CP_ERR_INVALID_ARG;
+  return cudaIpcCloseMemHandle(dptr) == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+}
+
+cp_status cp_peer_free(void* dptr) {
+  if (!dptr) return CP_ERR_INVALID_ARG;
+  return cudaFree(dptr) == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+}
+
+cp_status cp_ulysses_push_n(const void* const* srcs, void* const* dsts, int n_tensors, int rank, int degree, int B,
+                            int S, int H, int D, int direction, int elem_bytes, void* stream) {
+  NvtxRange nvtx_range("cp_ulysses_push_n");
+  if (degree < 1 || rank < 0 || rank >= degree || B < 0 || S < 0 || H < 0 || D < 0) return CP_ERR_INVALID_ARG;
+  if (direction != 0 && direction != 1) return CP_ERR_INVALID_ARG;
+  if (elem_bytes != 2 && elem_bytes != 4) return CP_ERR_UNSUPPORTED;
+  if (n_tensors < 1 || !srcs || !dsts) return CP_ERR_INVALID_ARG;
+  if (n_tensors > kPermuteMaxTensors || degree > kPeerMax) return CP_ERR_UNSUPPORTED;
+  if (S % degree != 0 || H % degree != 0) return CP_ERR_NOT_DIVISIBLE;
+  if (B == 0 || S == 0 || H == 0 || D == 0) return CP_OK;
+  const long long row_bytes = static_cast<long long>(H) * D * elem_bytes;
+  const long long piece_bytes = row_bytes / degree;
+  const int Sp = S / degree;
+  const long long total = static_cast<long long>(B) * Sp * row_bytes;  // bytes of every buffer
+  PushArgs a;
+  std::memset(&a, 0, sizeof(a));
+  uintptr_t bits = static_cast<uintptr_t>(piece_bytes);  // the widest vector dividing every offset
+  for (int t = 0; t < n_tensors; ++t) {
+    if (!srcs[t]) return CP_ERR_INVALID_ARG;
+    a.src[t] = srcs[t];
+    bits |= reinterpret_cast<uintptr_t>(srcs[t]);
+    for (int q = 0; q < degree; ++q) {
+      void* d = dsts[t * degree + q];
+      if (!d) return CP_ERR_INVALID_ARG;
+      a.dst[t][q] = d;
+      bits |= reinterpret_cast<uintptr_t>(d);
+    }
+  }
+  if (bits % elem_bytes) return CP_ERR_MISALIGNED;
+  // No destination may overlap a source or another destination.
+  for (int t = 0; t < n_tensors * degree; ++t) {
+    const char* d0 = static_cast<const char*>(dsts[t]);
+    for (int u = 0; u < n_tensors; ++u) {
+      const char* s0 = static_cast<const char*>(srcs[u]);
+      if (s0 < d0 + total && d0 < s0 + total) return CP_ERR_INVALID_ARG;
+    }
+    for (int u = 0; u < n_tensors * degree; ++u) {
+      const char* e0 = static_cast<const char*>(dsts[u]);
+      if (u != t && e0 < d0 + total && d0 < e0 + total) return CP_ERR_INVALID_ARG;
+    }
+  }
+  if (static_cast<long long>(n_tensors) * B > 65535 || row_bytes / 2 >= (1LL << 31)) return CP_ERR_UNSUPPORTED;
+  DeviceInfo* dev = nullptr;
+  cp_status st = device_info(&dev);
+  if (st != CP_OK) return st;
+  const int groups = (Sp + kPermuteRows - 1) / kPermuteRows;
+  const unsigned gy = static_cast<unsigned>(groups < 65535 ? groups : 65535);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  auto launch = [&](auto tag) {
+    using V = decltype(tag);
+    const int piece_vecs = static_cast<int>(piece_bytes / sizeof(V));
+    const int row_vecs = piece_vecs * degree;
+    const dim3 grid((row_vecs + kPermuteThreads - 1) / kPermuteThreads, gy, n_tensors * B);
+    ulysses_push_kernel<V><<<grid, kPermuteThreads, 0, cs>>>(a, rank, degree, B, Sp, piece_vecs, direction);
+  };
+  if (bits % 16 == 0)
+    launch(uint4{});
+  else if (bits % 8 == 0)
+    launch(uint2{});
+  else if (bits % 4 == 0)
+    launch(uint32_t{});
+  else
+    launch(uint16_t{});
+  return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+}
+
+cp_status cp_peer_barrier(void* const* signal_pads, int rank, int degree, unsigned int epoch, void* stream) {
+  NvtxRange nvtx_range("cp_peer_barrier");
+  if (degree < 1 || rank < 0 || rank >= degree || !signal_pads) return CP_ERR_INVALID_ARG;
+  if (degree > kPeerMax) return CP_ERR_UNSUPPORTED;
+  SignalTable t;
+  std::memset(&t, 0, sizeof(t));
+  for (int q = 0; q < degree; ++q) {
+    if (!signal_pads[q]) return CP_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(signal_pads[q]) & 3u) return CP_ERR_MISALIGNED;
+    t.pad[q] = static_cast<uint32_t*>(signal_pads[q]);
+  }
+  DeviceInfo* dev = nullptr;
+  cp_status st = device_info(&dev);
+  if (st != CP_OK) return st;
+  peer_barrier_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(t, rank, degree, epoch, dev->status);
+  return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+}
+
+cp_status cp_ring_fetch_block(void* dst, const void* src, int B, int rows, int H, int D, int dst_S, int dst_row0,
+                              int src_S, int src_row0, int elem_bytes, void* stream) {
+  NvtxRange nvtx_range("cp_ring_fetch_block");
+  if (B < 0 || rows < 0 || H < 0 || D < 0 || dst_row0 < 0 || src_row0 < 0) return CP_ERR_INVALID_ARG;
+  if (elem_bytes != 2 && elem_bytes != 4) return CP_ERR_UNSUPPORTED;
+  if (dst_row0 + static_cast<long long>(rows) > dst_S || src_row0 + static_cast<long long>(rows) > src_S)
+    return CP_ERR_INVALID_ARG;
+  if (B == 0 || rows == 0 || H == 0 || D == 0) return CP_OK;
+  if (!dst || !src) return CP_ERR_INVALID_ARG;
+  const size_t row = static_cast<size_t>(H) * D * elem_bytes;
+  char* d = static_cast<char*>(dst) + dst_row0 * row;
+  const char* s = static_cast<const char*>(src) + src_row0 * row;
+  const size_t dst_b = dst_S * row, src_b = src_S * row;
+  if (s < d + (B - 1) * dst_b + rows * row && d < s + (B - 1) * src_b + rows * row) return CP_ERR_INVALID_ARG;
+  return cudaMemcpy2DAsync(d, dst_b, s, src_b, rows * row, B, cudaMemcpyDefault, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? CP_OK
+             : CP_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -1,0 +1,128 @@
+// peer.cuh - the Ulysses exchange and the step barrier with one process per GPU.
+//
+// "Context parallelism", "Ulysses Attention": the two all-to-alls, done by pushes into
+// peer memory (buffers of the other GPUs mapped into this process with CUDA IPC).  Per
+// rank, with no leading degree dimension (P ranks, Sp = S/P tokens and Hp = H/P heads
+// per shard):
+//   sequence shard of rank r   X_r[b][s][h][:]    [B][Sp][H][D]
+//   head shard of rank q       Y_q[b][t][j][:]    [B][S][Hp][D]
+//   forward (direction 0): rank r stores, for every q,
+//       Y_q[b][r*Sp + s][j] = X_r[b][s][q*Hp + j]
+//   inverse (direction 1): rank r stores, for every p,
+//       X_p[b][s][r*Hp + j] = Y_r[b][p*Sp + s][j]
+// Run on every rank, the forward push fills exactly the layout of the single-GPU
+// exchange (ulysses_permute.cuh) split by rank.  Reads are local and writes go to the
+// owner, so every byte crosses NVLink once, as a store.
+//
+// The barrier orders the steps of one exchange across ranks: each rank writes the step's
+// epoch into its slot of every rank's signal pad, then waits, bounded, until every slot
+// of its own pad has reached the epoch.
+#pragma once
+
+#include <cstdint>
+
+#include "ptx_sm100.cuh"
+#include "ulysses_permute.cuh"
+
+namespace cpattn {
+
+constexpr int kPeerMax = 16;  // ranks in one exchange group
+
+struct PushArgs {
+  const void* src[kPermuteMaxTensors];
+  void* dst[kPermuteMaxTensors][kPeerMax];  // dst[t][q]: tensor t's buffer on rank q
+};
+
+// Work row (b, s) for s < Sp: P pieces of piece_vecs vectors, piece q going to (dir 0) or
+// coming from (dir 1) rank q.  grid.x covers the P*piece_vecs vectors of a work row,
+// grid.y groups of kPermuteRows rows (strided by gridDim.y), grid.z = tensor * B + b.
+template <typename V>
+__global__ void __launch_bounds__(kPermuteThreads)
+    ulysses_push_kernel(const __grid_constant__ PushArgs a, int rank, int P, int B, int Sp, int piece_vecs,
+                        int direction) {
+  const int row_vecs = P * piece_vecs;  // H*D elements of a sequence-shard row
+  const int i = blockIdx.x * kPermuteThreads + threadIdx.x;
+  if (i >= row_vecs) return;
+  const int q = i / piece_vecs;
+  const int w = i - q * piece_vecs;
+  const int n = blockIdx.z / B;
+  const int b = blockIdx.z - n * B;
+  const V* __restrict__ src = static_cast<const V*>(a.src[n]);
+  V* __restrict__ dst = static_cast<V*>(a.dst[n][q]);
+  const long long S = static_cast<long long>(Sp) * P;
+  // Vector offsets of work row 0 and the row strides, on the source and destination side.
+  const long long x0 = static_cast<long long>(b) * Sp * row_vecs;  // X row (b, 0)
+  long long s0, ss, d0, ds;
+  if (direction == 0) {
+    s0 = x0 + i;
+    ss = row_vecs;
+    d0 = (static_cast<long long>(b) * S + static_cast<long long>(rank) * Sp) * piece_vecs + w;
+    ds = piece_vecs;
+  } else {
+    s0 = (static_cast<long long>(b) * S + static_cast<long long>(q) * Sp) * piece_vecs + w;
+    ss = piece_vecs;
+    d0 = x0 + static_cast<long long>(rank) * piece_vecs + w;
+    ds = row_vecs;
+  }
+  const long long total = static_cast<long long>(B) * Sp * row_vecs;  // vectors of X_r and of Y_q alike
+  for (int sl0 = blockIdx.y * kPermuteRows; sl0 < Sp; sl0 += gridDim.y * kPermuteRows) {
+    V v[kPermuteRows];
+#pragma unroll
+    for (int r = 0; r < kPermuteRows; ++r) {
+      const int sl = sl0 + r;
+      if (sl < Sp && in_bounds(s0 + sl * ss, 1, total)) v[r] = src[s0 + sl * ss];
+    }
+#pragma unroll
+    for (int r = 0; r < kPermuteRows; ++r) {
+      const int sl = sl0 + r;
+      if (sl < Sp && in_bounds(d0 + sl * ds, 1, total)) dst[d0 + sl * ds] = v[r];
+    }
+  }
+  // The stores to other GPUs are performed before this kernel is seen as finished by the
+  // barrier that follows it on the stream.
+  __threadfence_system();
+}
+
+struct SignalTable {
+  uint32_t* pad[kPeerMax];  // pad[q]: rank q's signal pad, one word per rank
+};
+
+__device__ __forceinline__ void st_release_sys(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.sys.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_sys(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// One warp.  Lane q < P signals rank q (after a system-scope fence, so that this rank's
+// earlier writes, the stream's previous kernels included, are visible first), then lane q
+// waits for rank q's signal in this rank's pad.  Epochs increase by one per barrier and
+// are compared modulo 2^32.  A wait that runs past kWaitLimitCycles gives up and records
+// kDevTimeout in `status`; the kernel then returns.
+__global__ void __launch_bounds__(32)
+    peer_barrier_kernel(const __grid_constant__ SignalTable t, int rank, int P, uint32_t epoch, int* status) {
+  const int q = threadIdx.x;
+  if (q < P) {
+    __threadfence_system();
+    st_release_sys(t.pad[q] + rank, epoch);
+  }
+  bool ok = true;
+  if (q < P) {
+    const uint32_t* w = t.pad[rank] + q;
+    const long long t0 = clock64();
+    int polls = 0;
+    while (static_cast<int>(ld_acquire_sys(w) - epoch) < 0) {
+      if ((++polls & 15) == 0 && clock64() - t0 > kWaitLimitCycles) {
+        ok = false;
+        break;
+      }
+      __nanosleep(128);
+    }
+  }
+  if (!__all_sync(0xffffffffu, ok) && q == 0) atomicExch(status, kDevTimeout);
+}
+
+}  // namespace cpattn

@@ -19,7 +19,8 @@
  *   - LSE layout: float32 [B][H][Sq], natural logarithm.
  *   - Every pointer argument except chunk_bounds/bounds_out is a DEVICE pointer on
  *     the current CUDA device, owned by the caller; the library allocates no device
- *     memory and keeps no per-call state.  Device pointers must be 16-byte aligned.
+ *     memory and keeps no per-call state.  Device pointers must be 16-byte aligned,
+ *     except LSE arrays (float32, read and written one element at a time: 4 bytes).
  *   - stream: a cudaStream_t passed as void*; NULL means the legacy default stream.
  *     All calls are asynchronous on that stream; inputs must stay alive until the
  *     stream has executed the call.
@@ -63,6 +64,10 @@ typedef enum { CP_BF16 = 0, CP_F32 = 1 } cp_dtype;
 
 /* Largest number of K/V blocks a ring simulation or a merge accepts. */
 #define CP_MAX_CHUNKS 64
+
+/* Largest number of ranks in one peer exchange group, and the size of an IPC handle. */
+#define CP_PEER_MAX 16
+#define CP_IPC_HANDLE_BYTES 64
 
 /*
  * cp_attn_fwd - non-causal attention over one K/V block, returning its LSE.
@@ -282,6 +287,100 @@ CP_API cp_status cp_ulysses_permute(const void* src, void* dst, int degree, int 
  */
 CP_API cp_status cp_ulysses_permute_n(const void* const* srcs, void* const* dsts, int n_tensors, int degree,
                                int B, int S, int H, int D, int direction, int elem_bytes, void* stream);
+
+/*
+ * One process per GPU.  The calls below run the exchanges of "Context parallelism"
+ * ("Ring Attention", "Ulysses Attention", "Unified Attention") between real GPUs: peer
+ * buffers are plain device allocations shared with CUDA IPC; the Ulysses all-to-alls are
+ * pushes by this library's kernels into the other ranks' buffers; a ring rank fetches the
+ * other ranks' K/V blocks with the copy engines, so that the transfer overlaps the
+ * attention kernel (which holds every SM); a signal-pad barrier with a bounded wait
+ * orders the steps.  Process-group plumbing (who is rank q, exchanging the handles) is
+ * the caller's.
+ */
+
+/*
+ * cp_peer_alloc - a device buffer other processes can map.
+ *
+ * Allocates `bytes` (> 0) on the current device as its own allocation, zero-fills it
+ * (synchronously), and writes its CUDA IPC handle, CP_IPC_HANDLE_BYTES bytes, to the
+ * HOST buffer `handle`.  *dptr receives the device pointer (256-byte aligned); the caller
+ * owns it and releases it with cp_peer_free once every process that opened it has closed
+ * it.  Errors: bytes == 0 or a null pointer -> CP_ERR_INVALID_ARG; allocation or export
+ * failure -> CP_ERR_CUDA (nothing is left allocated).
+ */
+CP_API cp_status cp_peer_alloc(size_t bytes, void** dptr, void* handle);
+
+/*
+ * cp_peer_open - map another process's cp_peer_alloc buffer into this process.
+ *
+ * handle: HOST, CP_IPC_HANDLE_BYTES bytes from cp_peer_alloc in another process (CUDA
+ * does not open a handle in the process that made it).  Peer access is enabled on first
+ * use.  *dptr receives the mapping; release it with cp_peer_close.  Errors: null ->
+ * CP_ERR_INVALID_ARG; CUDA refused the handle -> CP_ERR_CUDA.
+ */
+CP_API cp_status cp_peer_open(const void* handle, void** dptr);
+
+/* cp_peer_close - unmap a cp_peer_open mapping.  cp_peer_free - free a cp_peer_alloc buffer.
+ * Both synchronous; null -> CP_ERR_INVALID_ARG; CUDA failure -> CP_ERR_CUDA. */
+CP_API cp_status cp_peer_close(void* dptr);
+CP_API cp_status cp_peer_free(void* dptr);
+
+/*
+ * cp_ulysses_push_n - this rank's half of a Ulysses all-to-all, pushed into peer buffers.
+ *
+ * Source: "Context parallelism", "Ulysses Attention".  P = degree ranks, Sp = S/P,
+ * Hp = H/P; per rank, sequence shard X [B][Sp][H][D] and head shard Y [B][S][Hp][D].
+ * direction 0 (first exchange): srcs[t] = this rank's X of tensor t;
+ *   dsts[t*P + q] = rank q's Y buffer of tensor t (a cp_peer_open mapping, or local for q
+ *   == rank); for every q: Y_q[b][rank*Sp + s][j][:] = X[b][s][q*Hp + j][:].
+ * direction 1 (second exchange): srcs[t] = this rank's Y; dsts[t*P + p] = rank p's X;
+ *   for every p: X_p[b][s][rank*Hp + j][:] = Y[b][p*Sp + s][j][:].
+ * Once every rank has pushed (and a barrier has passed), the buffers hold exactly what
+ * cp_ulysses_permute makes from the stacked shards.  A pure copy, bit-exact for any
+ * element type of elem_bytes (2 or 4) bytes.  srcs: HOST array of n_tensors pointers
+ * (1..8); dsts: HOST array of n_tensors*degree pointers; none overlapping another, all
+ * aligned to the element size (the copy uses the widest vector, up to 16 bytes, that
+ * divides every pointer and the piece of (H/P)*D elements).
+ * 1 <= degree <= CP_PEER_MAX, 0 <= rank < degree.
+ * The kernel ends with a system-scope fence; the writes are visible on the other GPUs
+ * once a cp_peer_barrier issued after it on the same stream has passed on both sides.
+ * Errors: S or H not divisible -> CP_ERR_NOT_DIVISIBLE; null, overlap, bad rank ->
+ * CP_ERR_INVALID_ARG; a pointer not aligned to the element -> CP_ERR_MISALIGNED; too
+ * many tensors or ranks ->
+ * CP_ERR_UNSUPPORTED.  Asynchronous on `stream`.
+ */
+CP_API cp_status cp_ulysses_push_n(const void* const* srcs, void* const* dsts, int n_tensors, int rank, int degree,
+                                   int B, int S, int H, int D, int direction, int elem_bytes, void* stream);
+
+/*
+ * cp_peer_barrier - all ranks of a group reach the same point of their streams.
+ *
+ * signal_pads: HOST array of degree pointers; signal_pads[q] = rank q's signal pad (at
+ * least degree 32-bit words of a cp_peer_alloc buffer, zero at first use, 4-byte aligned;
+ * this rank's own pad at index rank).  A one-warp kernel on `stream` first makes this
+ * rank's earlier writes visible system-wide, stores `epoch` into word `rank` of every
+ * pad, then waits until every word of its own pad has reached `epoch` (modulo 2^32:
+ * epochs start at 1 and grow by one per barrier; every rank passes the same sequence).
+ * The wait is bounded (about one second of SM clock): when it runs out the kernel records
+ * CP_ERR_TIMEOUT (read with cp_last_device_status) and returns, the context stays usable,
+ * and the group is to be treated as failed.  Errors: bad rank or null -> CP_ERR_INVALID_ARG;
+ * misaligned pad -> CP_ERR_MISALIGNED; degree > CP_PEER_MAX -> CP_ERR_UNSUPPORTED.
+ */
+CP_API cp_status cp_peer_barrier(void* const* signal_pads, int rank, int degree, unsigned int epoch, void* stream);
+
+/*
+ * cp_ring_fetch_block - copy rows [src_row0, src_row0+rows) of every batch of a
+ * [B][src_S][H][D] tensor to rows [dst_row0, ...) of a [B][dst_S][H][D] tensor.
+ *
+ * Source: "Context parallelism", "Ring Attention" (each rank sees every K/V block) and
+ * "Ring Anything Attention" (blocks of unequal length).  src may be another GPU's memory
+ * (a cp_peer_open mapping): the copy engines move it, so it overlaps a running kernel.
+ * Bit-exact.  elem_bytes 2 or 4.  Errors: rows outside either tensor, overlap, null ->
+ * CP_ERR_INVALID_ARG; CUDA failure -> CP_ERR_CUDA.  Asynchronous on `stream`.
+ */
+CP_API cp_status cp_ring_fetch_block(void* dst, const void* src, int B, int rows, int H, int D, int dst_S,
+                                     int dst_row0, int src_S, int src_row0, int elem_bytes, void* stream);
 
 /*
  * cp_ring_bounds - host-only helper: block bounds for a ring of n over S rows.

@@ -48,7 +48,7 @@ def test_sources_compile_and_export_header(tmp_path):
 
 
 def test_version_and_strings(lib):
-    assert lib.cp_version() == 100
+    assert lib.cp_version() == 101
     for code in (0, -1, -2, -3, -4, -5, -6, -7):
         assert binding.status_string(code).startswith("CP_")
 
@@ -74,6 +74,19 @@ def test_attn_fwd_rejects_before_launch(lib, args, want):
     *ptrs, B, H, Sq, Skv, D, scale, dt = args
     st = lib.cp_attn_fwd(*[ctypes.c_void_p(p) if p else None for p in ptrs], B, H, Sq, Skv, D, scale, dt, None)
     assert st == want
+
+
+def test_lse_needs_only_float_alignment(lib):
+    """LSE arrays are accessed one float at a time: 4-byte alignment is enough (a block's
+    LSE slice of an odd-length ring-anything block is not 16-byte aligned)."""
+    vp = ctypes.c_void_p
+    args = (vp(1 << 20), vp(2 << 20), vp(3 << 20), vp(4 << 20))
+    assert lib.cp_attn_fwd(*args, vp((5 << 20) + 2), 1, 2, 16, 16, 64, 0.1, 0, None) == I.CP_ERR_MISALIGNED
+    assert lib.cp_attn_fwd(*args, vp((5 << 20) + 4), 1, 2, 16, 16, 64, 0.1, 0, None) != I.CP_ERR_MISALIGNED
+    assert lib.cp_attn_merge(vp(1 << 20), vp((2 << 20) + 2), 2, vp(3 << 20), None, 1, 1, 1, 64, 0,
+                             None) == I.CP_ERR_MISALIGNED
+    assert lib.cp_attn_merge(vp(1 << 20), vp((2 << 20) + 4), 2, vp(3 << 20), vp((4 << 20) + 4), 1, 1, 1, 64, 0,
+                             None) != I.CP_ERR_MISALIGNED
 
 
 def test_merge_rejects(lib):
@@ -200,3 +213,47 @@ def test_pages_divisibility_rules(lib, row):
     else:  # ulysses: null pointers pass the divisibility check and stop at the pointer check
         st = lib.cp_ulysses_permute(None, None, degree, 1, tokens, heads, 128, 0, 2, None)
         assert st == (I.CP_ERR_INVALID_ARG if want == "ok" else I.CP_ERR_NOT_DIVISIBLE)
+
+
+def test_peer_calls_check_before_cuda(lib):
+    """The one-process-per-GPU calls reject bad arguments before any CUDA call."""
+    vp = ctypes.c_void_p
+    ptr = vp()
+    handle = ctypes.create_string_buffer(binding.CP_IPC_HANDLE_BYTES)
+    assert lib.cp_peer_alloc(0, ctypes.byref(ptr), handle) == I.CP_ERR_INVALID_ARG
+    assert lib.cp_peer_alloc(256, None, handle) == I.CP_ERR_INVALID_ARG
+    assert lib.cp_peer_open(None, ctypes.byref(ptr)) == I.CP_ERR_INVALID_ARG
+    assert lib.cp_peer_close(None) == I.CP_ERR_INVALID_ARG
+    assert lib.cp_peer_free(None) == I.CP_ERR_INVALID_ARG
+
+    src, dsts = (vp * 1)(1 << 20), (vp * 2)(2 << 20, 3 << 20)
+    push = lambda s, d, n, rank, deg, B, S, H, D, direc, eb: lib.cp_ulysses_push_n(  # noqa: E731
+        s, d, n, rank, deg, B, S, H, D, direc, eb, None)
+    assert push(src, dsts, 1, 2, 2, 1, 4, 4, 8, 0, 2) == I.CP_ERR_INVALID_ARG  # rank >= degree
+    assert push(src, dsts, 1, -1, 2, 1, 4, 4, 8, 0, 2) == I.CP_ERR_INVALID_ARG
+    assert push(src, dsts, 1, 0, 2, 1, 4, 4, 8, 2, 2) == I.CP_ERR_INVALID_ARG  # direction
+    assert push(src, dsts, 1, 0, 2, 1, 4, 4, 8, 0, 3) == I.CP_ERR_UNSUPPORTED  # element size
+    assert push(src, dsts, 9, 0, 2, 1, 4, 4, 8, 0, 2) == I.CP_ERR_UNSUPPORTED  # tensors
+    assert push(src, dsts, 1, 0, 17, 1, 34, 34, 8, 0, 2) == I.CP_ERR_UNSUPPORTED  # ranks
+    assert push(src, dsts, 1, 0, 2, 1, 5, 4, 8, 0, 2) == I.CP_ERR_NOT_DIVISIBLE
+    assert push(src, dsts, 1, 0, 2, 1, 4, 3, 8, 0, 2) == I.CP_ERR_NOT_DIVISIBLE
+    assert push(src, dsts, 1, 0, 2, 0, 4, 4, 8, 0, 2) == I.CP_OK  # empty: nothing to launch
+    assert push((vp * 1)((1 << 20) + 1), dsts, 1, 0, 2, 1, 4, 4, 8, 0, 2) == I.CP_ERR_MISALIGNED
+    assert push(src, (vp * 2)(2 << 20, (3 << 20) + 2), 1, 0, 2, 1, 4, 4, 8, 0, 4) == I.CP_ERR_MISALIGNED
+    assert push(src, (vp * 2)(1 << 20, 3 << 20), 1, 0, 2, 1, 4, 4, 8, 0, 2) == I.CP_ERR_INVALID_ARG  # overlap
+    assert push(src, (vp * 2)(2 << 20, 2 << 20), 1, 0, 2, 1, 4, 4, 8, 0, 2) == I.CP_ERR_INVALID_ARG
+    assert push(src, (vp * 2)(2 << 20, None), 1, 0, 2, 1, 4, 4, 8, 0, 2) == I.CP_ERR_INVALID_ARG
+
+    pads = (vp * 2)(1 << 20, 2 << 20)
+    assert lib.cp_peer_barrier(pads, 2, 2, 1, None) == I.CP_ERR_INVALID_ARG
+    assert lib.cp_peer_barrier(None, 0, 2, 1, None) == I.CP_ERR_INVALID_ARG
+    assert lib.cp_peer_barrier(pads, 0, 17, 1, None) == I.CP_ERR_UNSUPPORTED
+    assert lib.cp_peer_barrier((vp * 2)(1 << 20, None), 0, 2, 1, None) == I.CP_ERR_INVALID_ARG
+    assert lib.cp_peer_barrier((vp * 2)(1 << 20, (2 << 20) + 2), 0, 2, 1, None) == I.CP_ERR_MISALIGNED
+
+    fetch = lib.cp_ring_fetch_block
+    assert fetch(vp(1 << 20), vp(2 << 20), 1, 5, 2, 8, 4, 0, 8, 0, 2, None) == I.CP_ERR_INVALID_ARG  # past dst
+    assert fetch(vp(1 << 20), vp(2 << 20), 1, 5, 2, 8, 8, 0, 8, 4, 2, None) == I.CP_ERR_INVALID_ARG  # past src
+    assert fetch(vp(1 << 20), vp(2 << 20), 1, 1, 2, 8, 8, 0, 8, 0, 3, None) == I.CP_ERR_UNSUPPORTED
+    assert fetch(vp(1 << 20), vp(1 << 20), 1, 4, 2, 8, 8, 0, 8, 2, 2, None) == I.CP_ERR_INVALID_ARG  # overlap
+    assert fetch(None, None, 1, 0, 2, 8, 8, 0, 8, 0, 2, None) == I.CP_OK  # nothing to copy

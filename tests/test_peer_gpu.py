@@ -1,0 +1,143 @@
+"""The one-process-per-GPU exchange kernels on one GPU, with the ranks emulated by turns.
+
+cp_ulysses_push_n: every rank's push, launched one after another with each rank's
+"peer" buffers being local ones, must fill exactly the oracle's stacked exchange
+(bit-exact), in both directions.  cp_peer_barrier: passes when every signal is there
+(other ranks' signals written by the host), and runs out, bounded, reporting
+CP_ERR_TIMEOUT, when one never comes; the context stays usable.  cp_ring_fetch_block:
+a bit-exact row copy.  No kernel here waits on another kernel.
+"""
+
+import time
+
+import pytest
+import torch
+
+import oracle
+from context_attention_dit_b200 import binding
+from tests.gpu_util import cuda, qkv
+
+pytestmark = pytest.mark.gpu
+
+
+def _push_all(srcs, P, B, S, H, D, direction, dst_shape, dtype):
+    """Run every rank's push; returns the P destination buffers of every tensor."""
+    dsts = [[torch.zeros(dst_shape, dtype=dtype, device="cuda") for _ in range(P)] for _ in srcs]
+    stream = torch.cuda.current_stream().cuda_stream
+    for r in range(P):
+        binding.ulysses_push_n([s[r].data_ptr() for s in srcs], [[d.data_ptr() for d in row] for row in dsts], r, P,
+                               B, S, H, D, direction, srcs[0].element_size(), stream)
+    torch.cuda.synchronize()
+    return [torch.stack(row) for row in dsts]
+
+
+@pytest.mark.parametrize(
+    "P,B,S,H,D,dtype,n",
+    [
+        (2, 1, 256, 2, 64, torch.bfloat16, 1),
+        (8, 1, 4608, 24, 128, torch.bfloat16, 3),  # FLUX-like, Q/K/V in one launch
+        (4, 2, 4 * 37, 8, 128, torch.bfloat16, 3),  # ragged row groups
+        (3, 2, 9, 6, 5, torch.bfloat16, 1),  # odd piece size -> 2-byte vectors
+        (4, 2, 64, 8, 64, torch.float32, 2),
+        (16, 1, 160, 16, 128, torch.bfloat16, 1),  # the largest group
+        (1, 1, 33, 3, 128, torch.bfloat16, 1),  # degree 1: a local copy
+    ],
+)
+def test_push_fills_the_stacked_exchange(P, B, S, H, D, dtype, n):
+    g = torch.Generator().manual_seed(1000 + P * 10 + S)
+    xs = [torch.randn(P, B, S // P, H, D, generator=g).to(dtype) for _ in range(n)]
+    ys = _push_all([x.cuda() for x in xs], P, B, S, H, D, 0, (B, S, H // P, D), dtype)
+    for x, y in zip(xs, ys):
+        assert torch.equal(y.cpu(), oracle.ulysses_fwd(x, P))
+    back = _push_all(ys, P, B, S, H, D, 1, (B, S // P, H, D), dtype)
+    for x, b in zip(xs, back):
+        assert torch.equal(b.cpu(), x)
+
+
+def test_push_ulysses_attention_equals_unsplit():
+    """Ulysses attention by pushes (exchange, attention per head shard, inverse) is
+    bit-identical to attention of the unsplit sequence."""
+    P, B, S, H, D = 4, 1, 1024, 8, 128
+    q, k, v = cuda(*qkv(B, H, S, S, D, seed=7, rms=True))
+    shard = lambda x: x.reshape(B, P, S // P, H, D).permute(1, 0, 2, 3, 4).contiguous()  # noqa: E731
+    yq, yk, yv = _push_all([shard(q), shard(k), shard(v)], P, B, S, H, D, 0, (B, S, H // P, D), torch.bfloat16)
+    oh = torch.stack([binding.attn_fwd(yq[r], yk[r], yv[r], want_lse=False)[0] for r in range(P)])
+    (xo,) = _push_all([oh], P, B, S, H, D, 1, (B, S // P, H, D), torch.bfloat16)
+    full, _ = binding.attn_fwd(q, k, v, want_lse=False)
+    assert torch.equal(xo.permute(1, 0, 2, 3, 4).reshape(B, S, H, D), full)
+
+
+def test_push_rejects_bad_arguments():
+    x = torch.zeros(2, 8, 4, 64, dtype=torch.bfloat16, device="cuda")
+    y = [torch.zeros(2, 16, 2, 64, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    stream = torch.cuda.current_stream().cuda_stream
+    ptrs = [[t.data_ptr() for t in y]]
+    for rank, S, H, code in ((2, 16, 4, binding.CP_ERR_INVALID_ARG), (0, 15, 4, binding.CP_ERR_NOT_DIVISIBLE),
+                             (0, 16, 3, binding.CP_ERR_NOT_DIVISIBLE)):
+        with pytest.raises(binding.CpError) as e:
+            binding.ulysses_push_n([x.data_ptr()], ptrs, rank, 2, 2, S, H, 64, 0, 2, stream)
+        assert e.value.status == code
+    with pytest.raises(binding.CpError) as e:  # a destination overlapping the source
+        binding.ulysses_push_n([x.data_ptr()], [[x.data_ptr(), y[1].data_ptr()]], 0, 2, 2, 16, 4, 64, 0, 2, stream)
+    assert e.value.status == binding.CP_ERR_INVALID_ARG
+
+
+def _pads(n):
+    return [torch.zeros(binding.CP_PEER_MAX, dtype=torch.int32, device="cuda") for _ in range(n)]
+
+
+def test_barrier_passes_when_every_rank_signalled():
+    stream = torch.cuda.current_stream().cuda_stream
+    (pad,) = _pads(1)
+    for epoch in (1, 2, 3):  # degree 1: only its own signal
+        binding.peer_barrier([pad.data_ptr()], 0, epoch, stream)
+    assert binding.last_device_status() == binding.CP_OK
+    assert pad[0].item() == 3
+    # Degree 4, rank 2; ranks 0, 1, 3 have already signalled rank 2's pad (written here).
+    pads = _pads(4)
+    pads[2][:4] = torch.tensor([5, 5, 0, 6], dtype=torch.int32)
+    binding.peer_barrier([p.data_ptr() for p in pads], 2, 5, stream)
+    assert binding.last_device_status() == binding.CP_OK
+    for p in pads:  # rank 2's signal reached every pad
+        assert p[2].item() == 5
+    # Epochs compare modulo 2^32: rank 1 has already signalled epoch 1 (its counter
+    # wrapped past 0xFFFFFFFF), so rank 0's wait for 0xFFFFFFFF is over at once.
+    pads = _pads(2)
+    pads[0][1] = 1
+    binding.peer_barrier([p.data_ptr() for p in pads], 0, 0xFFFFFFFF, stream)
+    assert binding.last_device_status() == binding.CP_OK
+    assert pads[1][0].item() == -1  # 0xFFFFFFFF as int32
+
+
+def test_barrier_wait_runs_out_and_the_context_stays_usable():
+    stream = torch.cuda.current_stream().cuda_stream
+    pads = _pads(2)  # rank 1 never signals
+    t0 = time.time()
+    binding.peer_barrier([p.data_ptr() for p in pads], 0, 1, stream)
+    assert binding.last_device_status() == binding.CP_ERR_TIMEOUT
+    assert time.time() - t0 < 30
+    assert pads[1][0].item() == 1  # rank 0 still signalled before waiting
+    q, k, v = cuda(*qkv(1, 2, 256, 256, 64, seed=3))
+    o, _ = binding.attn_fwd(q, k, v)
+    assert binding.last_device_status() == binding.CP_OK
+    assert torch.isfinite(o.float()).all()
+
+
+@pytest.mark.parametrize("B,rows,H,D,dst_S,dst_row0,src_S,src_row0,dtype", [
+    (2, 1391, 24, 128, 4173, 1391, 1391, 0, torch.bfloat16),  # a ring-anything block into the gathered K
+    (1, 0, 4, 64, 10, 3, 10, 2, torch.bfloat16),
+    (3, 5, 3, 5, 7, 2, 9, 4, torch.float32),
+])
+def test_ring_fetch_block_copies_rows(B, rows, H, D, dst_S, dst_row0, src_S, src_row0, dtype):
+    g = torch.Generator().manual_seed(rows + dst_S)
+    src = torch.randn(B, src_S, H, D, generator=g).to(dtype).cuda()
+    dst = torch.zeros(B, dst_S, H, D, dtype=dtype, device="cuda")
+    binding.ring_fetch_block(dst.data_ptr(), src.data_ptr(), B, rows, H, D, dst_S, dst_row0, src_S, src_row0,
+                             src.element_size(), torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    want = torch.zeros_like(dst)
+    want[:, dst_row0:dst_row0 + rows] = src[:, src_row0:src_row0 + rows]
+    assert torch.equal(dst, want)
+    with pytest.raises(binding.CpError):
+        binding.ring_fetch_block(dst.data_ptr(), src.data_ptr(), B, dst_S + 1, H, D, dst_S, 0, src_S, 0,
+                                 src.element_size(), 0)
