@@ -42,6 +42,7 @@ EXPORTS = (
     "cp_debug_set_fault", "cp_last_device_status", "cp_status_string", "cp_version", "cp_usp_sim_workspace_size",
     "cp_usp_sim", "cp_ulysses_anything_permute", "cp_attn_merge_ulysses", "cp_peer_alloc", "cp_peer_open",
     "cp_peer_close", "cp_peer_free", "cp_ulysses_push_n", "cp_peer_barrier", "cp_ring_fetch_block",
+    "cp_ulysses_anything_push_n",
 )
 CP_PEER_MAX = 16
 CP_IPC_HANDLE_BYTES = 64
@@ -88,6 +89,9 @@ def load() -> ctypes.CDLL:
     lib.cp_peer_close.argtypes = [vp]
     lib.cp_peer_free.argtypes = [vp]
     lib.cp_ulysses_push_n.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), i, i, i, i, i, i, i, i, i, vp]
+    lib.cp_ulysses_anything_push_n.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), i, i, i, ip, ip, i, i, i, i,
+                                                i, vp]
+    lib.cp_ulysses_anything_push_n.restype = ctypes.c_int
     lib.cp_peer_barrier.argtypes = [ctypes.POINTER(vp), i, i, ctypes.c_uint, vp]
     lib.cp_ring_fetch_block.argtypes = [vp, vp, i, i, i, i, i, i, i, i, i, vp]
     lib.cp_debug_set_fault.argtypes = [i]
@@ -512,6 +516,24 @@ def ulysses_push_n(srcs: Sequence[int], dsts: Sequence[Sequence[int]], rank: int
     dp = (ctypes.c_void_p * (n * degree))(*[int(x) for row in dsts for x in row])
     _check(load().cp_ulysses_push_n(sp, dp, n, rank, degree, B, S, H, D, direction, elem_bytes, ctypes.c_void_p(stream)),
            "cp_ulysses_push_n")
+
+
+def ulysses_anything_push_n(srcs: Sequence[int], dsts: Sequence[Sequence[int]], rank: int,
+                            seq_bounds: Sequence[int], head_bounds: Sequence[int], B: int, H: int, D: int,
+                            direction: int, elem_bytes: int, stream: int):
+    """This rank's half of a Ulysses-Anything all-to-all (see cp_ulysses_anything_push_n)."""
+    degree = len(seq_bounds) - 1
+    n = len(srcs)
+    if degree < 1 or len(head_bounds) != degree + 1:
+        raise ValueError("seq_bounds and head_bounds need degree + 1 entries")
+    if n < 1 or len(dsts) != n or any(len(row) != degree for row in dsts):
+        raise ValueError("dsts needs one row of degree pointers per source")
+    sp = (ctypes.c_void_p * n)(*[int(x) for x in srcs])
+    dp = (ctypes.c_void_p * (n * degree))(*[int(x) for row in dsts for x in row])
+    sb = (ctypes.c_int * (degree + 1))(*[int(x) for x in seq_bounds])
+    hb = (ctypes.c_int * (degree + 1))(*[int(x) for x in head_bounds])
+    _check(load().cp_ulysses_anything_push_n(sp, dp, n, rank, degree, sb, hb, B, H, D, direction, elem_bytes,
+                                             ctypes.c_void_p(stream)), "cp_ulysses_anything_push_n")
 
 
 def peer_barrier(pads: Sequence[int], rank: int, epoch: int, stream: int):

@@ -715,6 +715,94 @@ cp_status cp_ulysses_push_n(const void* const* srcs, void* const* dsts, int n_te
   return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
 }
 
+cp_status cp_ulysses_anything_push_n(const void* const* srcs, void* const* dsts, int n_tensors, int rank, int degree,
+                                     const int* seq_bounds, const int* head_bounds, int B, int H, int D,
+                                     int direction, int elem_bytes, void* stream) {
+  NvtxRange nvtx_range("cp_ulysses_anything_push_n");
+  if (degree < 1 || rank < 0 || rank >= degree || B < 0 || H < 0 || D < 0 || !seq_bounds || !head_bounds)
+    return CP_ERR_INVALID_ARG;
+  if (direction != 0 && direction != 1) return CP_ERR_INVALID_ARG;
+  if (elem_bytes != 2 && elem_bytes != 4) return CP_ERR_UNSUPPORTED;
+  if (n_tensors < 1 || !srcs || !dsts) return CP_ERR_INVALID_ARG;
+  if (n_tensors > kPermuteMaxTensors || degree > kPeerMax) return CP_ERR_UNSUPPORTED;
+  if (seq_bounds[0] != 0 || head_bounds[0] != 0 || head_bounds[degree] != H) return CP_ERR_INVALID_ARG;
+  for (int i = 0; i < degree; ++i)
+    if (seq_bounds[i] > seq_bounds[i + 1] || head_bounds[i] > head_bounds[i + 1]) return CP_ERR_INVALID_ARG;
+  const int S = seq_bounds[degree];
+  const int Sr = seq_bounds[rank + 1] - seq_bounds[rank];
+  const int Hr = head_bounds[rank + 1] - head_bounds[rank];
+  // Rows this rank reads: its sequence shard (forward) or every token of its head shard.
+  if (B == 0 || H == 0 || D == 0 || (direction == 0 ? Sr : Hr) == 0) return CP_OK;
+  AnyPushArgs a;
+  std::memset(&a, 0, sizeof(a));
+  uintptr_t bits = static_cast<uintptr_t>(D) * elem_bytes;  // a vector never crosses a head
+  for (int t = 0; t < n_tensors; ++t) {
+    if (!srcs[t]) return CP_ERR_INVALID_ARG;
+    a.src[t] = srcs[t];
+    bits |= reinterpret_cast<uintptr_t>(srcs[t]);
+    for (int q = 0; q < degree; ++q) {
+      void* d = dsts[t * degree + q];
+      if (!d) return CP_ERR_INVALID_ARG;
+      a.dst[t][q] = d;
+      bits |= reinterpret_cast<uintptr_t>(d);
+    }
+  }
+  if (bits % elem_bytes) return CP_ERR_MISALIGNED;
+  // Byte extents: the source, and destination q of every tensor; none may overlap another.
+  const long long row = static_cast<long long>(D) * elem_bytes;
+  auto dst_bytes = [&](int q) {
+    return direction == 0 ? static_cast<long long>(B) * S * (head_bounds[q + 1] - head_bounds[q]) * row
+                          : static_cast<long long>(B) * (seq_bounds[q + 1] - seq_bounds[q]) * H * row;
+  };
+  const long long src_bytes = direction == 0 ? static_cast<long long>(B) * Sr * H * row
+                                             : static_cast<long long>(B) * S * Hr * row;
+  for (int t = 0; t < n_tensors * degree; ++t) {
+    const char* d0 = static_cast<const char*>(dsts[t]);
+    const long long dn = dst_bytes(t % degree);
+    for (int u = 0; u < n_tensors; ++u) {
+      const char* s0 = static_cast<const char*>(srcs[u]);
+      if (dn > 0 && s0 < d0 + dn && d0 < s0 + src_bytes) return CP_ERR_INVALID_ARG;
+    }
+    for (int u = 0; u < n_tensors * degree; ++u) {
+      const char* e0 = static_cast<const char*>(dsts[u]);
+      const long long en = dst_bytes(u % degree);
+      if (u != t && dn > 0 && en > 0 && e0 < d0 + dn && d0 < e0 + en) return CP_ERR_INVALID_ARG;
+    }
+  }
+  if (static_cast<long long>(n_tensors) * B * degree > 65535 || static_cast<long long>(H) * D >= (1LL << 31))
+    return CP_ERR_UNSUPPORTED;
+  DeviceInfo* dev = nullptr;
+  cp_status st = device_info(&dev);
+  if (st != CP_OK) return st;
+  int max_rows = Sr;
+  for (int i = 0; i <= degree; ++i) {
+    a.seq[i] = seq_bounds[i];
+    a.head[i] = head_bounds[i];
+    if (direction == 1 && i < degree && seq_bounds[i + 1] - seq_bounds[i] > max_rows)
+      max_rows = seq_bounds[i + 1] - seq_bounds[i];
+  }
+  const int groups = (max_rows + kPermuteRows - 1) / kPermuteRows;
+  const unsigned gy = static_cast<unsigned>(groups < 65535 ? groups : 65535);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  auto launch = [&](auto tag) {
+    using V = decltype(tag);
+    const int ve = static_cast<int>(sizeof(V)) / elem_bytes;
+    const long long row_vecs = static_cast<long long>(direction == 0 ? H : Hr) * D / ve;
+    const dim3 grid(static_cast<unsigned>((row_vecs + kPermuteThreads - 1) / kPermuteThreads), gy,
+                    n_tensors * B * (direction == 0 ? 1 : degree));
+    ulysses_anything_push_kernel<V><<<grid, kPermuteThreads, 0, cs>>>(a, rank, degree, B, H, D, ve, direction);
+  };
+  if (bits % 16 == 0)
+    launch(uint4{});
+  else if (bits % 8 == 0)
+    launch(uint2{});
+  else if (bits % 4 == 0)
+    launch(uint32_t{});
+  else
+    launch(uint16_t{});
+  return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+}
+
 cp_status cp_peer_barrier(void* const* signal_pads, int rank, int degree, unsigned int epoch, void* stream) {
   NvtxRange nvtx_range("cp_peer_barrier");
   if (degree < 1 || rank < 0 || rank >= degree || !signal_pads) return CP_ERR_INVALID_ARG;

@@ -83,6 +83,85 @@ __global__ void __launch_bounds__(kPermuteThreads)
   __threadfence_system();
 }
 
+// "Ulysses Anything Attention" with one process per GPU: shards of unequal size.  Sequence
+// shard p holds tokens [seq[p], seq[p+1]) and head shard q heads [head[q], head[q+1])
+// (either may be empty); per rank, X_r is [B][S_r][H][D] and Y_q is [B][S][H_q][D]:
+//   forward (direction 0): rank r stores, for every q,
+//       Y_q[b][seq[r] + s][j] = X_r[b][s][head[q] + j]
+//   inverse (direction 1): rank r stores, for every p,
+//       X_p[b][s][head[r] + j] = Y_r[b][seq[p] + s][j]
+struct AnyPushArgs {
+  const void* src[kPermuteMaxTensors];
+  void* dst[kPermuteMaxTensors][kPeerMax];
+  int seq[kPeerMax + 1];
+  int head[kPeerMax + 1];
+};
+
+// Forward: grid.x covers the vectors (VE elements, never crossing a head) of an X_r row,
+// grid.y groups of kPermuteRows rows of X_r (strided), grid.z = tensor * B + b.
+// Inverse: grid.x covers the vectors of a Y_r row, grid.y groups of rows of the
+// destination shard p, grid.z = (tensor * B + b) * P + p.
+template <typename V>
+__global__ void __launch_bounds__(kPermuteThreads)
+    ulysses_anything_push_kernel(const __grid_constant__ AnyPushArgs a, int rank, int P, int B, int H, int D, int VE,
+                                 int direction) {
+  const int S = a.seq[P];
+  const long long i = static_cast<long long>(blockIdx.x) * kPermuteThreads + threadIdx.x;
+  long long s0, ss, d0, ds, src_total, dst_total;  // vector offsets of row 0, row strides, extents
+  int rows;
+  V* __restrict__ dst;
+  const V* __restrict__ src;
+  if (direction == 0) {
+    if (i * VE >= static_cast<long long>(H) * D) return;
+    const int n = blockIdx.z / B, b = blockIdx.z - (blockIdx.z / B) * B;
+    const long long e = i * VE;
+    const int h = static_cast<int>(e / D);
+    int q = 0;
+    while (a.head[q + 1] <= h) ++q;  // the head group holding h (groups may be empty)
+    const long long Hq = a.head[q + 1] - a.head[q];
+    const int Sr = a.seq[rank + 1] - a.seq[rank];
+    rows = Sr;
+    src = static_cast<const V*>(a.src[n]);
+    dst = static_cast<V*>(a.dst[n][q]);
+    s0 = (static_cast<long long>(b) * Sr * H * D + e) / VE;
+    ss = static_cast<long long>(H) * D / VE;
+    d0 = ((static_cast<long long>(b) * S + a.seq[rank]) * Hq * D + e - static_cast<long long>(a.head[q]) * D) / VE;
+    ds = Hq * D / VE;
+    src_total = static_cast<long long>(B) * Sr * H * D / VE;
+    dst_total = static_cast<long long>(B) * S * Hq * D / VE;
+  } else {
+    const long long Hr = a.head[rank + 1] - a.head[rank];
+    if (i * VE >= Hr * D) return;
+    const int z = blockIdx.z / P, p = blockIdx.z - (blockIdx.z / P) * P;
+    const int n = z / B, b = z - (z / B) * B;
+    const long long e = i * VE;
+    const int Sp = a.seq[p + 1] - a.seq[p];
+    rows = Sp;
+    src = static_cast<const V*>(a.src[n]);
+    dst = static_cast<V*>(a.dst[n][p]);
+    s0 = ((static_cast<long long>(b) * S + a.seq[p]) * Hr * D + e) / VE;
+    ss = Hr * D / VE;
+    d0 = (static_cast<long long>(b) * Sp * H * D + static_cast<long long>(a.head[rank]) * D + e) / VE;
+    ds = static_cast<long long>(H) * D / VE;
+    src_total = static_cast<long long>(B) * S * Hr * D / VE;
+    dst_total = static_cast<long long>(B) * Sp * H * D / VE;
+  }
+  for (int sl0 = blockIdx.y * kPermuteRows; sl0 < rows; sl0 += gridDim.y * kPermuteRows) {
+    V v[kPermuteRows];
+#pragma unroll
+    for (int r = 0; r < kPermuteRows; ++r) {
+      const int sl = sl0 + r;
+      if (sl < rows && in_bounds(s0 + sl * ss, 1, src_total)) v[r] = src[s0 + sl * ss];
+    }
+#pragma unroll
+    for (int r = 0; r < kPermuteRows; ++r) {
+      const int sl = sl0 + r;
+      if (sl < rows && in_bounds(d0 + sl * ds, 1, dst_total)) dst[d0 + sl * ds] = v[r];
+    }
+  }
+  __threadfence_system();
+}
+
 struct SignalTable {
   uint32_t* pad[kPeerMax];  // pad[q]: rank q's signal pad, one word per rank
 };

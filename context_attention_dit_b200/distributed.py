@@ -288,38 +288,50 @@ class ContextParallel:
 
     # -- the step
 
-    def ring_lengths(self, local_len: int) -> List[int]:
-        """Every ring rank's block length, by ring index (host exchange over the ring group).
-        Uneven lengths are "Ring Anything Attention" and need ulysses_degree == 1."""
-        lens = [int(x) for x in exchange(int(local_len), self._pg["ring"])]
-        if self.U > 1 and len(set(lens)) > 1:
-            raise ValueError("uneven ring blocks need ulysses_degree == 1 (Ring Anything Attention)")
-        return lens
+    def shard_shapes(self, q) -> List[Tuple[int, int, int, int]]:
+        """Every rank's (B, S_local, H, D), by rank (a host exchange over the group).  All
+        ranks get the same list, so a mismatch raises on every rank alike."""
+        shapes = [tuple(int(x) for x in t) for t in exchange(tuple(q.shape), self.group)]
+        if len({(b, h, d) for b, _, h, d in shapes}) != 1:
+            raise ValueError(f"ranks disagree on batch, heads or head_dim: {shapes}")
+        return shapes
 
     def attention(self, q, k, v, scale: Optional[float] = None,
-                  ring_lengths: Optional[Sequence[int]] = None) -> torch.Tensor:
+                  seq_lengths: Optional[Sequence[int]] = None) -> torch.Tensor:
         """Attention of this rank's tokens over the whole sequence.
 
         q, k, v: this rank's sequence shard ``[B, S_local, H, D]``, contiguous bf16 on the
-        current device; H divisible by ulysses_degree when it is above 1.  ring_lengths:
-        every ring rank's block length (after the Ulysses exchange), by ring index; given,
-        it saves a host exchange per call, and it is only needed when the lengths differ
-        (ring anything, ulysses_degree == 1).  Returns ``[B, S_local, H, D]`` bf16.  With
-        ulysses_degree > 1 the result lives in a peer buffer that the next call
-        overwrites: copy it to keep it.
+        current device; the shards follow rank order along the sequence.  seq_lengths:
+        every rank's S_local, by rank; given, it saves a host exchange per call.  Returns
+        ``[B, S_local, H, D]`` bf16; with ulysses_degree > 1 the result lives in a peer
+        buffer that the next call overwrites (copy it to keep it).
+
+        Uneven shards follow the pages' variants table: with ring_degree 1 they are
+        "Ulysses Anything Attention" (S_local and H need not divide), with ulysses_degree 1
+        "Ring Anything Attention"; unified attention needs equal shards and H divisible by
+        ulysses_degree.
         """
         binding._check_qkv(q, k, v)
         if q.shape != k.shape:
             raise ValueError("query and key shards must have one shape")
         B, Sl, H, D = q.shape
         U, R = self.U, self.R
-        if U > 1 and H % U:
-            raise ValueError(f"heads {H} not divisible by ulysses_degree {U}")
         scale = float(D ** -0.5 if scale is None else scale)
+        if seq_lengths is None:
+            lengths = [s[1] for s in self.shard_shapes(q)]
+        else:
+            lengths = [int(x) for x in seq_lengths]
+        if len(lengths) != self.world or lengths[self.rank] != Sl:
+            raise ValueError(f"seq_lengths {lengths} do not hold this rank's {Sl} tokens at {self.rank}")
+        even = len(set(lengths)) == 1 and H % U == 0
+        if U > 1 and R > 1 and not even:
+            raise ValueError("unified attention needs equal shards and heads divisible by ulysses_degree")
         self.check_health()
         s = torch.cuda.current_stream(self.device)
         es = q.element_size()
         self.barrier("world")  # every rank is done with the previous step's buffers
+        if U > 1 and not even:
+            return self._ulysses_anything(q, k, v, lengths, scale)
         if U > 1:
             S_blk, Hh = Sl * U, H // U
             blk = B * S_blk * Hh * D * es
@@ -330,34 +342,47 @@ class ContextParallel:
             self.barrier("ulysses")
             qh, kh, vh = (self._view(b.local, (B, S_blk, Hh, D)) for b in bufs)
             kv_bufs = bufs[1:]
+            ring = [S_blk] * R
         else:
-            S_blk, Hh = Sl, H
             qh, kh, vh = q, k, v
             kv_bufs = None
+            ring = lengths  # U == 1: the ring group is the whole group, in rank order
         if R > 1:
-            if ring_lengths is not None:
-                lengths = [int(x) for x in ring_lengths]
-            elif U > 1:
-                lengths = [S_blk] * R
-            else:
-                lengths = self.ring_lengths(S_blk)
-            if len(lengths) != R or lengths[self.coord.ring_index] != S_blk:
-                raise ValueError(f"ring_lengths {lengths} do not hold this rank's {S_blk} rows at "
-                                 f"{self.coord.ring_index}")
             if kv_bufs is None:  # K/V into this rank's peer-visible buffers (sized alike on every rank)
-                kv_bufs = [self._buffer(n, B * max(lengths) * H * D * es) for n in ("rk", "rv")]
+                kv_bufs = [self._buffer(n, B * max(ring) * H * D * es) for n in ("rk", "rv")]
                 for src, b in ((k, kv_bufs[0]), (v, kv_bufs[1])):
-                    binding.ring_fetch_block(b.local, src.data_ptr(), B, S_blk, H, D, S_blk, 0, S_blk, 0, es,
-                                             s.cuda_stream)
+                    binding.ring_fetch_block(b.local, src.data_ptr(), B, Sl, H, D, Sl, 0, Sl, 0, es, s.cuda_stream)
             self.barrier("ring")  # every ring rank's K/V block is in place
-            oh = self._ring(qh, kh, vh, kv_bufs, lengths, scale)
+            oh = self._ring(qh, kh, vh, kv_bufs, ring, scale)
         else:
             oh, _ = binding.attn_fwd(qh, kh, vh, scale=scale, want_lse=False)
         if U == 1:
             return oh
         out = self._buffer("xo", B * Sl * H * D * es)
         binding.ulysses_push_n([oh.data_ptr()], [[out.ptrs[r] for r in self.coord.ulysses_ranks]],
-                               self.coord.ulysses_index, U, B, S_blk, H, D, 1, es, s.cuda_stream)
+                               self.coord.ulysses_index, U, B, Sl * U, H, D, 1, es, s.cuda_stream)
+        self.barrier("ulysses")
+        return self._view(out.local, (B, Sl, H, D))
+
+    def _ulysses_anything(self, q, k, v, lengths: List[int], scale: float) -> torch.Tensor:
+        """Ulysses with uneven sequence and head shards (ring_degree 1): sequence shards in
+        rank order, head shards as even as possible with the first ones larger."""
+        B, Sl, H, D = q.shape
+        U, me = self.U, self.rank
+        es = q.element_size()
+        s = torch.cuda.current_stream(self.device)
+        sb = block_bounds(lengths)
+        hb = binding.ring_bounds(H, U, anything=True)
+        S, Hr = sb[-1], hb[me + 1] - hb[me]
+        max_h = max(hb[i + 1] - hb[i] for i in range(U))
+        bufs = [self._buffer(n, B * S * max_h * D * es) for n in ("yq", "yk", "yv")]
+        binding.ulysses_anything_push_n([q.data_ptr(), k.data_ptr(), v.data_ptr()], [b.ptrs for b in bufs], me, sb,
+                                        hb, B, H, D, 0, es, s.cuda_stream)
+        self.barrier("ulysses")
+        qh, kh, vh = (self._view(b.local, (B, S, Hr, D)) for b in bufs)
+        oh, _ = binding.attn_fwd(qh, kh, vh, scale=scale, want_lse=False)
+        out = self._buffer("xo", B * max(lengths) * H * D * es)
+        binding.ulysses_anything_push_n([oh.data_ptr()], [out.ptrs], me, sb, hb, B, H, D, 1, es, s.cuda_stream)
         self.barrier("ulysses")
         return self._view(out.local, (B, Sl, H, D))
 

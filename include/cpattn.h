@@ -354,6 +354,27 @@ CP_API cp_status cp_ulysses_push_n(const void* const* srcs, void* const* dsts, i
                                    int B, int S, int H, int D, int direction, int elem_bytes, void* stream);
 
 /*
+ * cp_ulysses_anything_push_n - cp_ulysses_push_n for shards of unequal size.
+ *
+ * Source: "Context parallelism", "Ulysses Anything Attention" (sequence length and head
+ * count need not be divisible by ulysses_degree), with the layout of
+ * cp_ulysses_anything_permute: sequence shard p holds tokens [seq_bounds[p],
+ * seq_bounds[p+1]) and head shard q heads [head_bounds[q], head_bounds[q+1]); either may
+ * be empty.  Per rank: X_p [B][S_p][H][D], Y_q [B][S][H_q][D], S = seq_bounds[degree].
+ * direction 0: srcs[t] = this rank's X; dsts[t*P + q] = rank q's Y; for every q:
+ *   Y_q[b][seq_bounds[rank] + s][j][:] = X[b][s][head_bounds[q] + j][:].
+ * direction 1: srcs[t] = this rank's Y; dsts[t*P + p] = rank p's X; for every p:
+ *   X_p[b][s][head_bounds[rank] + j][:] = Y[b][seq_bounds[p] + s][j][:].
+ * seq_bounds, head_bounds: HOST int[degree+1], non-decreasing from 0 (head_bounds up to
+ * H).  Every rank's push together gives exactly cp_ulysses_anything_permute's shards.
+ * Other rules (pointers, alignment to the element, overlap, ordering by cp_peer_barrier,
+ * errors) as cp_ulysses_push_n; bad bounds -> CP_ERR_INVALID_ARG.
+ */
+CP_API cp_status cp_ulysses_anything_push_n(const void* const* srcs, void* const* dsts, int n_tensors, int rank,
+                                            int degree, const int* seq_bounds, const int* head_bounds, int B, int H,
+                                            int D, int direction, int elem_bytes, void* stream);
+
+/*
  * cp_peer_barrier - all ranks of a group reach the same point of their streams.
  *
  * signal_pads: HOST array of degree pointers; signal_pads[q] = rank q's signal pad (at

@@ -257,3 +257,24 @@ def test_peer_calls_check_before_cuda(lib):
     assert fetch(vp(1 << 20), vp(2 << 20), 1, 1, 2, 8, 8, 0, 8, 0, 3, None) == I.CP_ERR_UNSUPPORTED
     assert fetch(vp(1 << 20), vp(1 << 20), 1, 4, 2, 8, 8, 0, 8, 2, 2, None) == I.CP_ERR_INVALID_ARG  # overlap
     assert fetch(None, None, 1, 0, 2, 8, 8, 0, 8, 0, 2, None) == I.CP_OK  # nothing to copy
+
+
+def test_anything_push_checks_before_cuda(lib):
+    vp = ctypes.c_void_p
+    src, dsts = (vp * 1)(1 << 20), (vp * 2)(2 << 20, 3 << 20)
+    sb, hb = _bounds(0, 3, 5), _bounds(0, 2, 3)
+    call = lambda s, d, rank, sbd, hbd, H, direc=0, eb=2: lib.cp_ulysses_anything_push_n(  # noqa: E731
+        s, d, 1, rank, 2, sbd, hbd, 1, H, 8, direc, eb, None)
+    assert call(src, dsts, 2, sb, hb, 3) == I.CP_ERR_INVALID_ARG  # rank >= degree
+    assert call(src, dsts, 0, None, hb, 3) == I.CP_ERR_INVALID_ARG
+    assert call(src, dsts, 0, _bounds(1, 3, 5), hb, 3) == I.CP_ERR_INVALID_ARG  # bounds must start at 0
+    assert call(src, dsts, 0, _bounds(0, 4, 3), hb, 3) == I.CP_ERR_INVALID_ARG  # decreasing
+    assert call(src, dsts, 0, sb, hb, 4) == I.CP_ERR_INVALID_ARG  # head bounds must end at H
+    assert call(src, dsts, 0, sb, hb, 3, 2) == I.CP_ERR_INVALID_ARG  # direction
+    assert call(src, dsts, 0, sb, hb, 3, 0, 3) == I.CP_ERR_UNSUPPORTED
+    assert call(src, dsts, 0, _bounds(0, 0, 5), hb, 3) == I.CP_OK  # this rank holds no tokens: nothing to push
+    assert call(src, dsts, 1, sb, _bounds(0, 3, 3), 3, 1) == I.CP_OK  # this rank holds no heads
+    assert call((vp * 1)((1 << 20) + 1), dsts, 0, sb, hb, 3) == I.CP_ERR_MISALIGNED
+    assert call(src, (vp * 2)(1 << 20, 3 << 20), 0, sb, hb, 3) == I.CP_ERR_INVALID_ARG  # overlap
+    assert call(src, (vp * 2)(None, 3 << 20), 0, sb, hb, 3) == I.CP_ERR_INVALID_ARG
+    assert lib.cp_ulysses_anything_push_n(src, dsts, 1, 0, 17, sb, hb, 1, 3, 8, 0, 2, None) == I.CP_ERR_UNSUPPORTED

@@ -122,6 +122,8 @@ def _run(U, R, B, H, D, lens, oracle_check=False):
     "U,R,B,H,D,lens,oracle_check",
     [
         (2, 1, 1, 4, 128, [512, 512], True),  # Ulysses
+        (3, 1, 1, 5, 128, [101, 100, 99], True),  # Ulysses anything: uneven tokens, 5 heads over 3
+        (3, 1, 2, 2, 64, [64, 64, 63], False),  # Ulysses anything with an empty head shard
         (2, 1, 1, 24, 128, [2304, 2304], False),  # Ulysses on the FLUX-like shape
         (1, 2, 2, 3, 128, [301, 300], True),  # ring anything: uneven blocks
         (1, 3, 1, 2, 64, [384, 384, 384], False),  # ring of three

@@ -54,6 +54,43 @@ def test_push_fills_the_stacked_exchange(P, B, S, H, D, dtype, n):
         assert torch.equal(b.cpu(), x)
 
 
+ANYTHING = [  # (P, B, S, H, D, dtype): uneven sequence and head shards, empty ones included
+    (4, 1, 4481, 24, 128, torch.bfloat16),  # FLUX-1008^2 over 4 ranks
+    (5, 1, 4608, 24, 128, torch.bfloat16),  # 24 heads over 5 ranks
+    (3, 2, 10, 7, 3, torch.bfloat16),  # odd head_dim -> 2-byte vectors
+    (5, 1, 4, 3, 64, torch.float32),  # more ranks than tokens and heads: empty shards
+    (2, 2, 9, 1, 64, torch.bfloat16),
+]
+
+
+@pytest.mark.parametrize("P,B,S,H,D,dtype", ANYTHING)
+def test_anything_push_fills_the_oracle_shards(P, B, S, H, D, dtype):
+    g = torch.Generator().manual_seed(2000 + P * 10 + S)
+    x = torch.randn(B, S, H, D, generator=g).to(dtype)
+    sb = binding.ring_bounds(S, P, anything=True)
+    hb = binding.ring_bounds(H, P, anything=True)
+    xs = [x[:, sb[p]:sb[p + 1]].contiguous() for p in range(P)]
+    want = oracle.ulysses_anything_fwd(xs, sb, hb)
+    stream = torch.cuda.current_stream().cuda_stream
+    # Separate allocations stand in for the ranks' buffers (sizes differ per shard).
+    xg = [t.cuda() for t in xs]
+    ys = [torch.zeros(B, S, hb[q + 1] - hb[q], D, dtype=dtype, device="cuda") for q in range(P)]
+    ptr = lambda t: t.data_ptr() if t.numel() else 16  # noqa: E731  (an empty shard is never touched)
+    for r in range(P):
+        binding.ulysses_anything_push_n([ptr(xg[r])], [[ptr(y) for y in ys]], r, sb, hb, B, H, D, 0,
+                                        x.element_size(), stream)
+    torch.cuda.synchronize()
+    for q in range(P):
+        assert torch.equal(ys[q].cpu(), torch.as_tensor(want[q]))
+    back = [torch.zeros(B, sb[p + 1] - sb[p], H, D, dtype=dtype, device="cuda") for p in range(P)]
+    for r in range(P):
+        binding.ulysses_anything_push_n([ptr(ys[r])], [[ptr(t) for t in back]], r, sb, hb, B, H, D, 1,
+                                        x.element_size(), stream)
+    torch.cuda.synchronize()
+    for p in range(P):
+        assert torch.equal(back[p].cpu(), xs[p])
+
+
 def test_push_ulysses_attention_equals_unsplit():
     """Ulysses attention by pushes (exchange, attention per head shard, inverse) is
     bit-identical to attention of the unsplit sequence."""
