@@ -321,6 +321,17 @@ def run_ours(args):
     any_bytes = 2 * xa.numel() * xa.element_size()
     del xa, ya
 
+    # One process per GPU: every rank's push of Q/K/V (cp_ulysses_push_n), the ranks taken
+    # in turn on this GPU with local buffers for their peers' (NVLink is not measured here).
+    def push_all():
+        st = torch.cuda.current_stream().cuda_stream
+        for r in range(P):
+            binding.ulysses_push_n([xq[r].data_ptr(), xk[r].data_ptr(), xv[r].data_ptr()],
+                                   [[t[p].data_ptr() for p in range(P)] for t in (yq, yk, yv)], r, P, B, S, H, D,
+                                   0, 2, st)
+
+    push_ms = timed_ms(push_all)
+
     # End to end through the public API with host buffers (pinned), per step: H2D of the
     # sequence-sharded Q/K/V, the hot path, D2H of O.  Steps are pipelined over three
     # streams with two buffer slots, as a serving loop would run them: the upload of step
@@ -425,6 +436,8 @@ def run_ours(args):
                 **usp,
                 "anything_permute_flux1008_p4_ms": round(any_ms, 4),
                 "anything_permute_flux1008_p4_gbs": round(any_bytes / (any_ms * 1e-3) / 1e9, 1),
+                "push_qkv_8_ranks_by_turns_ms": round(push_ms, 4),
+                "push_qkv_8_ranks_by_turns_gbs": round(perm_bytes / (push_ms * 1e-3) / 1e9, 1),
             },
             "e2e": {"value": round(world * flop / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
