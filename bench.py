@@ -566,6 +566,13 @@ def run_profile_case(args):
             xs = [t.view(B, P, S // P, H, D).permute(1, 0, 2, 3, 4).contiguous() for t in (q, k, v)]
             ys = binding.ulysses_permute_n(xs, P, 0)
             binding.ulysses_permute(ys[0], P, 1)
+        elif case == "push":  # every rank's Q/K/V push, ranks by turns, local buffers for the peers'
+            xs = [t.view(B, P, S // P, H, D).permute(1, 0, 2, 3, 4).contiguous() for t in (q, k, v)]
+            ys = [torch.empty(P, B, S, H // P, D, dtype=torch.bfloat16, device="cuda") for _ in range(3)]
+            st = torch.cuda.current_stream().cuda_stream
+            for r in range(P):
+                binding.ulysses_push_n([x[r].data_ptr() for x in xs], [[y[p].data_ptr() for p in range(P)] for y in ys],
+                                       r, P, B, S, H, D, 0, 2, st)
     torch.cuda.synchronize()
     assert binding.last_device_status() == 0
     print(f"profile case {case} x{args.profile_reps} batch {B}: ok")
@@ -580,7 +587,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-budget", type=float, default=90.0)
-    ap.add_argument("--profile-case", choices=["attn_ring1", "attn_ring8", "merge", "permute"], default=None)
+    ap.add_argument("--profile-case", choices=["attn_ring1", "attn_ring8", "merge", "permute", "push"], default=None)
     ap.add_argument("--profile-batch", type=int, default=2)
     ap.add_argument("--profile-reps", type=int, default=3)
     args = ap.parse_args()
