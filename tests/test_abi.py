@@ -35,6 +35,19 @@ def test_exported_symbols_in_dynamic_table():
     assert set(declared_functions()) <= exported
 
 
+def test_in_tree_debug_library_is_current():
+    """The debug build that travels with the tree exports every declared entry point (a
+    stale one would fail only on the GPU)."""
+    import subprocess
+
+    from context_attention_dit_b200 import build
+
+    if not os.path.exists(build.LIB_DEBUG):
+        pytest.skip("debug library not built")
+    out = subprocess.run(["nm", "-D", "--defined-only", build.LIB_DEBUG], capture_output=True, text=True).stdout
+    assert set(declared_functions()) <= set(re.findall(r"\b(cp_[a-z0-9_]+)\b", out))
+
+
 def test_sources_compile_and_export_header(tmp_path):
     """The current sources (not only the in-tree binary) build for sm_100a and export every
     declared entry point."""
