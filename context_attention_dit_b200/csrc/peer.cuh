@@ -78,9 +78,8 @@ __global__ void __launch_bounds__(kPermuteThreads)
       if (sl < Sp && in_bounds(d0 + sl * ds, 1, total)) dst[d0 + sl * ds] = v[r];
     }
   }
-  // The stores to other GPUs are performed before this kernel is seen as finished by the
-  // barrier that follows it on the stream.
-  __threadfence_system();
+  // No fence here: a kernel's stores, to other GPUs included, are performed when it
+  // completes, before the barrier kernel that follows it on the stream signals anyone.
 }
 
 // "Ulysses Anything Attention" with one process per GPU: shards of unequal size.  Sequence
@@ -159,7 +158,6 @@ __global__ void __launch_bounds__(kPermuteThreads)
       if (sl < rows && in_bounds(d0 + sl * ds, 1, dst_total)) dst[d0 + sl * ds] = v[r];
     }
   }
-  __threadfence_system();
 }
 
 struct SignalTable {

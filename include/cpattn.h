@@ -343,8 +343,9 @@ CP_API cp_status cp_peer_free(void* dptr);
  * aligned to the element size (the copy uses the widest vector, up to 16 bytes, that
  * divides every pointer and the piece of (H/P)*D elements).
  * 1 <= degree <= CP_PEER_MAX, 0 <= rank < degree.
- * The kernel ends with a system-scope fence; the writes are visible on the other GPUs
- * once a cp_peer_barrier issued after it on the same stream has passed on both sides.
+ * The writes are performed at the other GPUs when the kernel completes; they are visible
+ * to a peer's later work once a cp_peer_barrier issued after it on the same stream has
+ * passed on both sides.
  * Errors: S or H not divisible -> CP_ERR_NOT_DIVISIBLE; null, overlap, bad rank ->
  * CP_ERR_INVALID_ARG; a pointer not aligned to the element -> CP_ERR_MISALIGNED; too
  * many tensors or ranks ->
