@@ -42,7 +42,7 @@ EXPORTS = (
     "cp_debug_set_fault", "cp_last_device_status", "cp_status_string", "cp_version", "cp_usp_sim_workspace_size",
     "cp_usp_sim", "cp_ulysses_anything_permute", "cp_attn_merge_ulysses", "cp_peer_alloc", "cp_peer_open",
     "cp_peer_close", "cp_peer_free", "cp_ulysses_push_n", "cp_peer_barrier", "cp_ring_fetch_block",
-    "cp_ulysses_anything_push_n",
+    "cp_ulysses_anything_push_n", "cp_attn_merge_push",
 )
 CP_PEER_MAX = 16
 CP_IPC_HANDLE_BYTES = 64
@@ -92,6 +92,8 @@ def load() -> ctypes.CDLL:
     lib.cp_ulysses_anything_push_n.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), i, i, i, ip, ip, i, i, i, i,
                                                 i, vp]
     lib.cp_ulysses_anything_push_n.restype = ctypes.c_int
+    lib.cp_attn_merge_push.argtypes = [vp, vp, i, ctypes.POINTER(vp), i, i, i, i, i, i, i, vp]
+    lib.cp_attn_merge_push.restype = ctypes.c_int
     lib.cp_peer_barrier.argtypes = [ctypes.POINTER(vp), i, i, ctypes.c_uint, vp]
     lib.cp_ring_fetch_block.argtypes = [vp, vp, i, i, i, i, i, i, i, i, i, vp]
     lib.cp_debug_set_fault.argtypes = [i]
@@ -534,6 +536,23 @@ def ulysses_anything_push_n(srcs: Sequence[int], dsts: Sequence[Sequence[int]], 
     hb = (ctypes.c_int * (degree + 1))(*[int(x) for x in head_bounds])
     _check(load().cp_ulysses_anything_push_n(sp, dp, n, rank, degree, sb, hb, B, H, D, direction, elem_bytes,
                                              ctypes.c_void_p(stream)), "cp_ulysses_anything_push_n")
+
+
+def attn_merge_push(partials, lses, peer_outs: Sequence[int], shard: int, out_dtype=torch.bfloat16):
+    """Merge this rank's head-shard partials ``[n, B, S, H/P, D]`` (LSEs ``[n, B, H/P, S]``)
+    and store every merged row into its owner's sequence shard ``[B, S/P, H, D]``:
+    ``peer_outs[p]`` is rank p's (see cp_attn_merge_push)."""
+    if partials.dtype != torch.float32 or lses.dtype != torch.float32:
+        raise ValueError("partials and lses must be float32")
+    if not (partials.is_cuda and lses.is_cuda and partials.is_contiguous() and lses.is_contiguous()):
+        raise ValueError("partials and lses must be contiguous CUDA tensors")
+    n, B, S, Hp, D = partials.shape
+    if tuple(lses.shape) != (n, B, Hp, S):
+        raise ValueError(f"incompatible shapes partials{tuple(partials.shape)} lses{tuple(lses.shape)}")
+    P = len(peer_outs)
+    po = (ctypes.c_void_p * P)(*[int(x) for x in peer_outs])
+    _check(load().cp_attn_merge_push(_ptr(partials), _ptr(lses), n, po, shard, P, B, S, Hp * P, D,
+                                     _out_code(out_dtype), ctypes.c_void_p(_stream(partials))), "cp_attn_merge_push")
 
 
 def peer_barrier(pads: Sequence[int], rank: int, epoch: int, stream: int):

@@ -24,7 +24,7 @@ using namespace cpattn;
 
 static_assert(kMaxChunks == CP_MAX_CHUNKS, "chunk limit mismatch");
 static_assert(kDevTimeout == CP_ERR_TIMEOUT && kDevBounds == CP_ERR_BOUNDS, "device status codes mismatch");
-static_assert(kPeerMax == CP_PEER_MAX, "peer limit mismatch");
+static_assert(kPeerMax == CP_PEER_MAX && kPeerMergeMax == CP_PEER_MAX, "peer limit mismatch");
 static_assert(sizeof(cudaIpcMemHandle_t) == CP_IPC_HANDLE_BYTES, "IPC handle size mismatch");
 
 namespace {
@@ -193,7 +193,8 @@ cp_status launch_attn(const void* q, const void* k, const void* v, const int* bo
 }
 
 cp_status launch_merge(const float* partials, const float* lses, int n, void* out, float* out_lse, int B, int H,
-                       int Sq, int D, cp_dtype out_dtype, cudaStream_t stream, int ulysses_p = 0, int ulysses_b = 0) {
+                       int Sq, int D, cp_dtype out_dtype, cudaStream_t stream, int ulysses_p = 0, int ulysses_b = 0,
+                       const MergePeers* peers = nullptr, int shard = 0) {
   const long long rows = static_cast<long long>(B) * H * Sq;
   const long long part_stride = rows * D;
   const long long lse_stride = rows;
@@ -204,12 +205,18 @@ cp_status launch_merge(const float* partials, const float* lses, int n, void* ou
   const size_t smem = static_cast<size_t>(n) * H * ST * sizeof(float);
   if (smem > 48 * 1024) return CP_ERR_UNSUPPORTED;
   const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(B));
+  const MergePeers none{};
   auto launch = [&](auto kernel) {
     kernel<<<grid, kMergeThreads, smem, stream>>>(partials, lses, n, out, out_lse, H, Sq, ST, part_stride, lse_stride,
-                                                  ulysses_p, ulysses_b);
+                                                  ulysses_p, ulysses_b, peers ? *peers : none, shard);
   };
   const bool bf16 = out_dtype == CP_BF16;
-  if (ulysses_p > 0) {
+  if (peers) {
+    if (D == 128)
+      bf16 ? launch(lse_merge_kernel<128, true, false, true>) : launch(lse_merge_kernel<128, false, false, true>);
+    else
+      bf16 ? launch(lse_merge_kernel<64, true, false, true>) : launch(lse_merge_kernel<64, false, false, true>);
+  } else if (ulysses_p > 0) {
     if (D == 128)
       bf16 ? launch(lse_merge_kernel<128, true, true>) : launch(lse_merge_kernel<128, false, true>);
     else
@@ -801,6 +808,29 @@ cp_status cp_ulysses_anything_push_n(const void* const* srcs, void* const* dsts,
   else
     launch(uint16_t{});
   return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+}
+
+cp_status cp_attn_merge_push(const float* partials, const float* lses, int n_chunks, void* const* peer_outs,
+                             int shard, int degree, int B, int S, int H, int D, cp_dtype out_dtype, void* stream) {
+  NvtxRange nvtx_range("cp_attn_merge_push");
+  if (degree < 1 || shard < 0 || shard >= degree || B < 0 || S < 0 || H < 0) return CP_ERR_INVALID_ARG;
+  if (degree > kPeerMergeMax) return CP_ERR_UNSUPPORTED;
+  if (S % degree != 0 || H % degree != 0) return CP_ERR_NOT_DIVISIBLE;
+  if (n_chunks < 1 || n_chunks > CP_MAX_CHUNKS) return n_chunks < 1 ? CP_ERR_INVALID_ARG : CP_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128) return CP_ERR_UNSUPPORTED;
+  if (out_dtype != CP_BF16 && out_dtype != CP_F32) return CP_ERR_INVALID_ARG;
+  if (B == 0 || H == 0 || S == 0) return CP_OK;
+  if (!partials || !lses || !peer_outs) return CP_ERR_INVALID_ARG;
+  if (!aligned16(partials) || !aligned4(lses)) return CP_ERR_MISALIGNED;
+  MergePeers peers{};
+  for (int q = 0; q < degree; ++q) {
+    if (!peer_outs[q]) return CP_ERR_INVALID_ARG;
+    if (!aligned16(peer_outs[q])) return CP_ERR_MISALIGNED;
+    peers.out[q] = peer_outs[q];
+  }
+  if (B > 65535) return CP_ERR_UNSUPPORTED;
+  return launch_merge(partials, lses, n_chunks, nullptr, nullptr, B, H / degree, S, D, out_dtype,
+                      static_cast<cudaStream_t>(stream), degree, B, &peers, shard);
 }
 
 cp_status cp_peer_barrier(void* const* signal_pads, int rank, int degree, unsigned int epoch, void* stream) {

@@ -23,16 +23,26 @@
 namespace cpattn {
 
 constexpr int kMergeThreads = 256;
+constexpr int kPeerMergeMax = 16;  // ranks of a Ulysses group
 
 // kUlysses: the partials are those of attention on Ulysses head shards (batch P*Bs, H heads
 // per shard, shard p = heads [p*H, (p+1)*H) of P*H), and the merged output goes straight to
 // the sequence-sharded layout of the inverse exchange, [P][Bs][Sq/P][P*H][D] (the merge and
 // the second all-to-all of "Ulysses Attention" in one pass), with the LSE as [Bs][P*H][Sq].
-template <int D, bool kOutBf16, bool kUlysses>
+//
+// kPeer (one process per GPU): the partials are this rank's head shard only (batch Bs, H
+// heads, shard index `shard` of P), and the merged row of token s goes to rank s/(Sq/P)'s
+// sequence shard, peer_out[s/(Sq/P)] as [Bs][Sq/P][P*H][D], over peer memory: the merge and
+// this rank's half of the second all-to-all in one kernel.  No LSE is written.
+struct MergePeers {
+  void* out[kPeerMergeMax];
+};
+
+template <int D, bool kOutBf16, bool kUlysses, bool kPeer = false>
 __global__ void __launch_bounds__(kMergeThreads)
     lse_merge_kernel(const float* __restrict__ partials, const float* __restrict__ lses, int n, void* __restrict__ out,
                      float* __restrict__ out_lse, int H, int Sq, int ST, long long part_stride, long long lse_stride,
-                     int P, int Bs) {
+                     int P, int Bs, const __grid_constant__ MergePeers peers = MergePeers{}, int shard = 0) {
   constexpr int kVec = D / 32;  // floats per lane: 4 (D=128) or 2 (D=64)
   constexpr float kLog2e = 1.4426950408889634f;
   constexpr float kLn2 = 0.69314718055994530942f;
@@ -69,6 +79,7 @@ __global__ void __launch_bounds__(kMergeThreads)
     const long long eoff = row * D + lane * kVec;
     long long ooff = eoff;                                                 // output element
     long long lrow = (static_cast<long long>(b) * H + h) * Sq + s;        // [B][H][Sq]
+    void* dst = out;
     if (kUlysses) {
       const int p = b / Bs, bs = b - (b / Bs) * Bs;  // head shard, batch
       const int Sp = Sq / P;
@@ -76,6 +87,12 @@ __global__ void __launch_bounds__(kMergeThreads)
       ooff = (((static_cast<long long>(ps) * Bs + bs) * Sp + sl) * (static_cast<long long>(P) * H) + p * H + h) * D +
              lane * kVec;
       lrow = (static_cast<long long>(bs) * P * H + p * H + h) * Sq + s;
+    }
+    if (kPeer) {
+      const int Sp = Sq / P;
+      const int ps = s / Sp, sl = s - (s / Sp) * Sp;  // owner rank, token within its shard
+      dst = peers.out[ps];
+      ooff = ((static_cast<long long>(b) * Sp + sl) * (static_cast<long long>(P) * H) + shard * H + h) * D + lane * kVec;
     }
 #ifdef CP_DEBUG
     // The row's partial vectors (every block), its output vector and its LSE.  The whole
@@ -88,15 +105,15 @@ __global__ void __launch_bounds__(kMergeThreads)
     if (M == -INFINITY) {  // every block empty
       if (kOutBf16) {
         if (kVec == 4)
-          *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out) + ooff) = make_uint2(0u, 0u);
+          *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(dst) + ooff) = make_uint2(0u, 0u);
         else
-          *reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(out) + ooff) = 0u;
+          *reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(dst) + ooff) = 0u;
       } else {
-        float* o = static_cast<float*>(out) + ooff;
+        float* o = static_cast<float*>(dst) + ooff;
 #pragma unroll
         for (int i = 0; i < kVec; ++i) o[i] = 0.f;
       }
-      if (lane == 0 && out_lse) out_lse[lrow] = -INFINITY;
+      if (!kPeer && lane == 0 && out_lse) out_lse[lrow] = -INFINITY;
       continue;
     }
     // exp(x - M) = 2^((x - M) * log2 e); exp(-inf) = 0 for empty blocks.
@@ -127,19 +144,19 @@ __global__ void __launch_bounds__(kMergeThreads)
       }
     }
     if (kOutBf16) {
-      __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out) + ooff;
+      __nv_bfloat16* o = static_cast<__nv_bfloat16*>(dst) + ooff;
       if (kVec == 4)
         *reinterpret_cast<uint2*>(o) = make_uint2(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]));
       else
         *reinterpret_cast<uint32_t*>(o) = pack_bf16x2(acc[0], acc[1]);
     } else {
-      float* o = static_cast<float*>(out) + ooff;
+      float* o = static_cast<float*>(dst) + ooff;
       if (kVec == 4)
         *reinterpret_cast<float4*>(o) = make_float4(acc[0], acc[1], acc[2], acc[3]);
       else
         *reinterpret_cast<float2*>(o) = make_float2(acc[0], acc[1]);
     }
-    if (lane == 0 && out_lse) out_lse[lrow] = L2 * kLn2;
+    if (!kPeer && lane == 0 && out_lse) out_lse[lrow] = L2 * kLn2;
   }
 }
 

@@ -14,7 +14,9 @@ Data moves through this package's library only:
 * a ring rank fetches the other ring ranks' K/V blocks with ``cp_ring_fetch_block`` (the
   copy engines, on a side stream, one event per block), and attends each block as soon as
   it has landed: its own block first, while the others are still in flight;
-* the blocks' fp32 partials are merged by their LSEs (``cp_attn_merge``);
+* the blocks' fp32 partials are merged by their LSEs (``cp_attn_merge``); in unified
+  attention the merge stores each row straight into its owner's sequence shard
+  (``cp_attn_merge_push``: the merge and the second all-to-all in one kernel);
 * ``cp_peer_barrier`` orders the steps, with a bounded device-side wait.
 
 ``torch.distributed`` (NCCL on GPUs, gloo in the CPU tests) carries the plumbing only: the
@@ -353,9 +355,17 @@ class ContextParallel:
                 for src, b in ((k, kv_bufs[0]), (v, kv_bufs[1])):
                     binding.ring_fetch_block(b.local, src.data_ptr(), B, Sl, H, D, Sl, 0, Sl, 0, es, s.cuda_stream)
             self.barrier("ring")  # every ring rank's K/V block is in place
-            oh = self._ring(qh, kh, vh, kv_bufs, ring, scale)
-        else:
-            oh, _ = binding.attn_fwd(qh, kh, vh, scale=scale, want_lse=False)
+            partials, lses = self._ring(qh, kh, vh, kv_bufs, ring, scale)
+            if U == 1:
+                return binding.attn_merge(partials, lses)[0]
+            # Unified: the merge stores every row straight into its owner's sequence shard
+            # (the second all-to-all fused into the merge).
+            out = self._buffer("xo", B * Sl * H * D * es)
+            binding.attn_merge_push(partials, lses, [out.ptrs[r] for r in self.coord.ulysses_ranks],
+                                    self.coord.ulysses_index)
+            self.barrier("ulysses")
+            return self._view(out.local, (B, Sl, H, D))
+        oh, _ = binding.attn_fwd(qh, kh, vh, scale=scale, want_lse=False)
         if U == 1:
             return oh
         out = self._buffer("xo", B * Sl * H * D * es)
@@ -386,8 +396,9 @@ class ContextParallel:
         self.barrier("ulysses")
         return self._view(out.local, (B, Sl, H, D))
 
-    def _ring(self, qh, kh, vh, kv_bufs, lengths: List[int], scale: float) -> torch.Tensor:
-        """Ring attention of the local queries over every ring rank's K/V block."""
+    def _ring(self, qh, kh, vh, kv_bufs, lengths: List[int], scale: float):
+        """Ring attention of the local queries over every ring rank's K/V block: returns
+        the blocks' fp32 partials and LSEs, in block order."""
         B, Sq, Hh, D = qh.shape
         R, me = self.R, self.coord.ring_index
         es = qh.element_size()
@@ -422,5 +433,4 @@ class ContextParallel:
                 kc = land_k[offs[c]: offs[c + 1]].view(B, n, Hh, D)
                 vc = land_v[offs[c]: offs[c + 1]].view(B, n, Hh, D)
             binding.attn_fwd(qh, kc, vc, scale=scale, out_dtype=torch.float32, out=partials[c], lse=lses[c])
-        out, _ = binding.attn_merge(partials, lses)
-        return out
+        return partials, lses

@@ -376,6 +376,27 @@ CP_API cp_status cp_ulysses_anything_push_n(const void* const* srcs, void* const
                                             int D, int direction, int elem_bytes, void* stream);
 
 /*
+ * cp_attn_merge_push - LSE merge of this rank's head-shard partials, each merged row
+ * stored straight into its owner's sequence shard over peer memory.
+ *
+ * Source: "Context parallelism", "Unified Attention" (ring attention on the Ulysses head
+ * shards, then the second all-to-all) and "Ring Attention" (blocks merged through their
+ * LSEs, as cp_attn_merge).  P = degree ranks of a Ulysses group; this rank holds head
+ * shard `shard` (heads [shard*H/P, (shard+1)*H/P)) for all S tokens.
+ * partials: fp32 [n_chunks][B][S][H/P][D]; lses: fp32 [n_chunks][B][H/P][S].
+ * peer_outs: HOST array of P device pointers, peer_outs[p] = rank p's sequence shard
+ * [B][S/P][H][D] (a cp_peer_open mapping, or local for p == shard): the merged row of
+ * token s, head j goes to peer_outs[s/(S/P)][b][s%(S/P)][shard*H/P + j].  No LSE is
+ * written.  The merge arithmetic is cp_attn_merge's, so the rows are bit-identical to it.
+ * Ordering as cp_ulysses_push_n (a cp_peer_barrier after it).  Errors: as cp_attn_merge;
+ * S or H not divisible -> CP_ERR_NOT_DIVISIBLE; bad shard -> CP_ERR_INVALID_ARG;
+ * degree > CP_PEER_MAX -> CP_ERR_UNSUPPORTED.
+ */
+CP_API cp_status cp_attn_merge_push(const float* partials, const float* lses, int n_chunks, void* const* peer_outs,
+                                    int shard, int degree, int B, int S, int H, int D, cp_dtype out_dtype,
+                                    void* stream);
+
+/*
  * cp_peer_barrier - all ranks of a group reach the same point of their streams.
  *
  * signal_pads: HOST array of degree pointers; signal_pads[q] = rank q's signal pad (at

@@ -291,3 +291,21 @@ def test_anything_push_checks_before_cuda(lib):
     assert call(src, (vp * 2)(1 << 20, 3 << 20), 0, sb, hb, 3) == I.CP_ERR_INVALID_ARG  # overlap
     assert call(src, (vp * 2)(None, 3 << 20), 0, sb, hb, 3) == I.CP_ERR_INVALID_ARG
     assert lib.cp_ulysses_anything_push_n(src, dsts, 1, 0, 17, sb, hb, 1, 3, 8, 0, 2, None) == I.CP_ERR_UNSUPPORTED
+
+
+def test_merge_push_checks_before_cuda(lib):
+    vp = ctypes.c_void_p
+    outs = (vp * 2)(3 << 20, 4 << 20)
+    call = lambda parts, outs_, shard, deg, S, H, D=64, n=2, dt=0: lib.cp_attn_merge_push(  # noqa: E731
+        parts, vp(2 << 20), n, outs_, shard, deg, 1, S, H, D, dt, None)
+    assert call(vp(1 << 20), outs, 2, 2, 8, 4) == I.CP_ERR_INVALID_ARG  # shard >= degree
+    assert call(vp(1 << 20), outs, 0, 17, 34, 34) == I.CP_ERR_UNSUPPORTED
+    assert call(vp(1 << 20), outs, 0, 2, 7, 4) == I.CP_ERR_NOT_DIVISIBLE
+    assert call(vp(1 << 20), outs, 0, 2, 8, 3) == I.CP_ERR_NOT_DIVISIBLE
+    assert call(vp(1 << 20), outs, 0, 2, 8, 4, D=96) == I.CP_ERR_UNSUPPORTED
+    assert call(vp(1 << 20), outs, 0, 2, 8, 4, n=0) == I.CP_ERR_INVALID_ARG
+    assert call(vp(1 << 20), outs, 0, 2, 8, 4, dt=5) == I.CP_ERR_INVALID_ARG
+    assert call(vp((1 << 20) + 4), outs, 0, 2, 8, 4) == I.CP_ERR_MISALIGNED
+    assert call(vp(1 << 20), (vp * 2)(3 << 20, (4 << 20) + 8), 0, 2, 8, 4) == I.CP_ERR_MISALIGNED
+    assert call(vp(1 << 20), (vp * 2)(3 << 20, None), 0, 2, 8, 4) == I.CP_ERR_INVALID_ARG
+    assert call(None, None, 0, 2, 0, 4) == I.CP_OK  # empty

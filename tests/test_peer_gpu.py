@@ -119,6 +119,28 @@ def test_push_rejects_bad_arguments():
     assert e.value.status == binding.CP_ERR_INVALID_ARG
 
 
+@pytest.mark.parametrize("P,n,B,S,H,D,dtype", [
+    (8, 8, 1, 4608, 24, 128, torch.bfloat16),  # the bench's merge, one rank's head shard at a time
+    (2, 3, 2, 100, 4, 64, torch.float32),
+    (4, 2, 1, 36, 8, 128, torch.bfloat16),
+])
+def test_merge_push_equals_fused_merge(P, n, B, S, H, D, dtype):
+    """Each rank's merge of its head shard, stored into the ranks' sequence shards, gives
+    exactly cp_attn_merge_ulysses's output (bit for bit)."""
+    g = torch.Generator().manual_seed(3000 + S)
+    Hp = H // P
+    parts = torch.randn(n, P * B, S, Hp, D, generator=g).cuda()
+    lses = (4 * torch.randn(n, P * B, Hp, S, generator=g)).cuda()
+    lses[0, :, :, :3] = -float("inf")  # a block with no keys for some rows
+    want, _ = binding.attn_merge_ulysses(parts, lses, P, out_dtype=dtype)
+    outs = [torch.full((B, S // P, H, D), float("nan"), dtype=dtype, device="cuda") for _ in range(P)]
+    for u in range(P):
+        binding.attn_merge_push(parts[:, u * B:(u + 1) * B].contiguous(), lses[:, u * B:(u + 1) * B].contiguous(),
+                                [o.data_ptr() for o in outs], u, out_dtype=dtype)
+    torch.cuda.synchronize()
+    assert torch.equal(torch.stack(outs), want)
+
+
 def _pads(n):
     return [torch.zeros(binding.CP_PEER_MAX, dtype=torch.int32, device="cuda") for _ in range(n)]
 
