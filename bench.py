@@ -175,7 +175,7 @@ def run_ours(args):
     import torch.distributed as dist
 
     from context_attention_dit_b200 import binding
-    from context_attention_dit_b200.inputs import WORKLOADS, even_bounds, sha256
+    from context_attention_dit_b200.inputs import WORKLOADS, bounds_from_sizes, even_bounds, sha256
 
     world, rank, local = dist_setup()
     torch.cuda.set_device(local)
@@ -321,6 +321,27 @@ def run_ours(args):
     any_bytes = 2 * xa.numel() * xa.element_size()
     del xa, ya
 
+    # The other workloads (parity cases, reported beside the bench line, not as it): ring /
+    # ring-anything attention, blocks + LSE merge (cp_ring_sim), over each of their splits.
+    other_configs = {}
+    for name in ("tiny_s256_d64", "uneven_s4173_ring3", "video_s32760_ring4"):
+        wl = WORKLOADS[name]
+        cq, ck, cv = (t.to(dev) for t in wl.qkv())
+        for i, sizes in enumerate(wl.splits):
+            bnd = bounds_from_sizes(sizes)
+            cws = torch.empty(max(binding.ring_workspace_size(len(sizes), wl.B, wl.H, wl.S, wl.D), 1),
+                              dtype=torch.uint8, device=dev)
+            co = torch.empty_like(cq)
+            cl = torch.empty((wl.B, wl.H, wl.S), dtype=torch.float32, device=dev)
+            ms = timed_ms(lambda: binding.ring_sim(cq, ck, cv, bnd, scale=wl.scale, workspace=cws, out=co,
+                                                   out_lse=cl), reps=5 if wl.S > 20000 else 20)
+            key = name if len(wl.splits) == 1 else f"{name}_split{i}"
+            other_configs[key] = {"blocks": list(sizes), "ms": round(ms, 4),
+                                  "tflops": round(wl.flop / (ms * 1e-3) / 1e12, 2)}
+            del cws, co, cl
+        del cq, ck, cv
+    torch.cuda.empty_cache()
+
     # One process per GPU: every rank's push of Q/K/V (cp_ulysses_push_n), the ranks taken
     # in turn on this GPU with local buffers for their peers' (NVLink is not measured here).
     def push_all():
@@ -444,6 +465,7 @@ def run_ours(args):
                 "push_qkv_8_ranks_by_turns_ms": round(push_ms, 4),
                 "push_qkv_8_ranks_by_turns_gbs": round(perm_bytes / (push_ms * 1e-3) / 1e9, 1),
             },
+            "other_configs": other_configs,
             "e2e": {"value": round(world * flop / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
             "gpu_launches": launches_per_step * args.steps,
