@@ -94,7 +94,7 @@ def load() -> ctypes.CDLL:
     lib.cp_ulysses_anything_push_n.restype = ctypes.c_int
     lib.cp_attn_merge_push.argtypes = [vp, vp, i, ctypes.POINTER(vp), i, i, i, i, i, i, i, vp]
     lib.cp_attn_merge_push.restype = ctypes.c_int
-    lib.cp_peer_barrier.argtypes = [ctypes.POINTER(vp), i, i, ctypes.c_uint, vp]
+    lib.cp_peer_barrier.argtypes = [ctypes.POINTER(vp), i, i, ctypes.c_uint, ctypes.c_uint, vp]
     lib.cp_ring_fetch_block.argtypes = [vp, vp, i, i, i, i, i, i, i, i, i, vp]
     lib.cp_debug_set_fault.argtypes = [i]
     lib.cp_debug_set_fault.restype = ctypes.c_int
@@ -555,12 +555,13 @@ def attn_merge_push(partials, lses, peer_outs: Sequence[int], shard: int, out_dt
                                      _out_code(out_dtype), ctypes.c_void_p(_stream(partials))), "cp_attn_merge_push")
 
 
-def peer_barrier(pads: Sequence[int], rank: int, epoch: int, stream: int):
-    """Signal every rank's pad and wait (bounded) for every rank's signal (see cp_peer_barrier)."""
+def peer_barrier(pads: Sequence[int], rank: int, epoch: int, stream: int, timeout_ms: int = 1000):
+    """Signal every rank's pad and wait, at most ``timeout_ms``, for every rank's signal
+    (see cp_peer_barrier)."""
     n = len(pads)
     pp = (ctypes.c_void_p * n)(*[int(x) for x in pads])
-    _check(load().cp_peer_barrier(pp, rank, n, ctypes.c_uint(epoch & 0xFFFFFFFF), ctypes.c_void_p(stream)),
-           "cp_peer_barrier")
+    _check(load().cp_peer_barrier(pp, rank, n, ctypes.c_uint(epoch & 0xFFFFFFFF), ctypes.c_uint(int(timeout_ms)),
+                                  ctypes.c_void_p(stream)), "cp_peer_barrier")
 
 
 def ring_fetch_block(dst: int, src: int, B: int, rows: int, H: int, D: int, dst_S: int, dst_row0: int, src_S: int,

@@ -833,7 +833,8 @@ cp_status cp_attn_merge_push(const float* partials, const float* lses, int n_chu
                       static_cast<cudaStream_t>(stream), degree, B, &peers, shard);
 }
 
-cp_status cp_peer_barrier(void* const* signal_pads, int rank, int degree, unsigned int epoch, void* stream) {
+cp_status cp_peer_barrier(void* const* signal_pads, int rank, int degree, unsigned int epoch,
+                          unsigned int timeout_ms, void* stream) {
   NvtxRange nvtx_range("cp_peer_barrier");
   if (degree < 1 || rank < 0 || rank >= degree || !signal_pads) return CP_ERR_INVALID_ARG;
   if (degree > kPeerMax) return CP_ERR_UNSUPPORTED;
@@ -847,7 +848,9 @@ cp_status cp_peer_barrier(void* const* signal_pads, int rank, int degree, unsign
   DeviceInfo* dev = nullptr;
   cp_status st = device_info(&dev);
   if (st != CP_OK) return st;
-  peer_barrier_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(t, rank, degree, epoch, dev->status);
+  const uint64_t limit_ns = static_cast<uint64_t>(timeout_ms ? timeout_ms : 1000u) * 1000000ull;
+  peer_barrier_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(t, rank, degree, epoch, limit_ns,
+                                                                      dev->status);
   return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
 }
 

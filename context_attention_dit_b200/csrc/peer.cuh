@@ -174,13 +174,20 @@ __device__ __forceinline__ uint32_t ld_acquire_sys(const uint32_t* p) {
   return v;
 }
 
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
 // One warp.  Lane q < P signals rank q (after a system-scope fence, so that this rank's
 // earlier writes, the stream's previous kernels included, are visible first), then lane q
 // waits for rank q's signal in this rank's pad.  Epochs increase by one per barrier and
-// are compared modulo 2^32.  A wait that runs past kWaitLimitCycles gives up and records
-// kDevTimeout in `status`; the kernel then returns.
+// are compared modulo 2^32.  A wait that runs past `limit_ns` of wall-clock time (the
+// global timer) gives up and records kDevTimeout in `status`; the kernel then returns.
 __global__ void __launch_bounds__(32)
-    peer_barrier_kernel(const __grid_constant__ SignalTable t, int rank, int P, uint32_t epoch, int* status) {
+    peer_barrier_kernel(const __grid_constant__ SignalTable t, int rank, int P, uint32_t epoch, uint64_t limit_ns,
+                        int* status) {
   const int q = threadIdx.x;
   if (q < P) {
     __threadfence_system();
@@ -189,10 +196,10 @@ __global__ void __launch_bounds__(32)
   bool ok = true;
   if (q < P) {
     const uint32_t* w = t.pad[rank] + q;
-    const long long t0 = clock64();
+    const uint64_t t0 = global_ns();
     int polls = 0;
     while (static_cast<int>(ld_acquire_sys(w) - epoch) < 0) {
-      if ((++polls & 15) == 0 && clock64() - t0 > kWaitLimitCycles) {
+      if ((++polls & 15) == 0 && global_ns() - t0 > limit_ns) {
         ok = false;
         break;
       }

@@ -188,12 +188,15 @@ class ContextParallel:
 
     Every rank calls the constructor and every method in the same order (the buffers are
     allocated collectively).  ``barrier="device"`` orders steps with ``cp_peer_barrier``
-    (stream-ordered, no host sync); ``barrier="host"`` synchronises the stream and calls
-    the process group's barrier instead.
+    (stream-ordered, no host sync), whose wait gives up after ``barrier_timeout_ms``: ranks
+    are driven by their hosts, so the limit must cover the host-side skew between ranks.
+    A barrier that gave up leaves the step's outputs undefined; :meth:`check_device`
+    reports it.  ``barrier="host"`` synchronises the stream and calls the process group's
+    barrier instead.
     """
 
     def __init__(self, ulysses_degree: int = 1, ring_degree: int = 1, group=None, barrier: str = "device",
-                 monitor: Optional[HealthMonitor] = None):
+                 monitor: Optional[HealthMonitor] = None, barrier_timeout_ms: int = 30000):
         if barrier not in ("device", "host"):
             raise ValueError("barrier must be 'device' or 'host'")
         self.group = group
@@ -206,6 +209,7 @@ class ContextParallel:
         self.U, self.R = int(ulysses_degree), int(ring_degree)
         self.coord = mesh_coord(self.rank, self.U, self.R)
         self.barrier_mode = barrier
+        self.barrier_timeout_ms = int(barrier_timeout_ms)
         self.monitor = monitor
         self.device = torch.device("cuda", torch.cuda.current_device())
         # Sub-groups for the host barrier: every rank creates every group, in one order.
@@ -243,7 +247,8 @@ class ContextParallel:
         self._epoch[name] += 1
         off = _GROUPS.index(name) * _PAD_WORDS * 4
         pads = [self._pads.ptrs[r] + off for r in members]
-        binding.peer_barrier(pads, members.index(self.rank), self._epoch[name], s.cuda_stream)
+        binding.peer_barrier(pads, members.index(self.rank), self._epoch[name], s.cuda_stream,
+                             self.barrier_timeout_ms)
 
     def _retire(self, bufs: Sequence[_PeerBuffer]):
         """Free peer buffers: every rank stops using them, unmaps the others', then frees

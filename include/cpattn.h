@@ -405,12 +405,15 @@ CP_API cp_status cp_attn_merge_push(const float* partials, const float* lses, in
  * rank's earlier writes visible system-wide, stores `epoch` into word `rank` of every
  * pad, then waits until every word of its own pad has reached `epoch` (modulo 2^32:
  * epochs start at 1 and grow by one per barrier; every rank passes the same sequence).
- * The wait is bounded (about one second of SM clock): when it runs out the kernel records
- * CP_ERR_TIMEOUT (read with cp_last_device_status) and returns, the context stays usable,
- * and the group is to be treated as failed.  Errors: bad rank or null -> CP_ERR_INVALID_ARG;
- * misaligned pad -> CP_ERR_MISALIGNED; degree > CP_PEER_MAX -> CP_ERR_UNSUPPORTED.
+ * The wait is bounded by timeout_ms of wall-clock time (the GPU's global timer; 0 means
+ * 1000 ms): when it runs out the kernel records CP_ERR_TIMEOUT (read with
+ * cp_last_device_status) and returns, the context stays usable, and the group is to be
+ * treated as failed; whatever the stream runs after a timed-out barrier works on data
+ * that may not have arrived.  Errors: bad rank or null -> CP_ERR_INVALID_ARG; misaligned
+ * pad -> CP_ERR_MISALIGNED; degree > CP_PEER_MAX -> CP_ERR_UNSUPPORTED.
  */
-CP_API cp_status cp_peer_barrier(void* const* signal_pads, int rank, int degree, unsigned int epoch, void* stream);
+CP_API cp_status cp_peer_barrier(void* const* signal_pads, int rank, int degree, unsigned int epoch,
+                                 unsigned int timeout_ms, void* stream);
 
 /*
  * cp_ring_fetch_block - copy rows [src_row0, src_row0+rows) of every batch of a

@@ -258,11 +258,11 @@ def test_peer_calls_check_before_cuda(lib):
     assert push(src, (vp * 2)(2 << 20, None), 1, 0, 2, 1, 4, 4, 8, 0, 2) == I.CP_ERR_INVALID_ARG
 
     pads = (vp * 2)(1 << 20, 2 << 20)
-    assert lib.cp_peer_barrier(pads, 2, 2, 1, None) == I.CP_ERR_INVALID_ARG
-    assert lib.cp_peer_barrier(None, 0, 2, 1, None) == I.CP_ERR_INVALID_ARG
-    assert lib.cp_peer_barrier(pads, 0, 17, 1, None) == I.CP_ERR_UNSUPPORTED
-    assert lib.cp_peer_barrier((vp * 2)(1 << 20, None), 0, 2, 1, None) == I.CP_ERR_INVALID_ARG
-    assert lib.cp_peer_barrier((vp * 2)(1 << 20, (2 << 20) + 2), 0, 2, 1, None) == I.CP_ERR_MISALIGNED
+    assert lib.cp_peer_barrier(pads, 2, 2, 1, 0, None) == I.CP_ERR_INVALID_ARG
+    assert lib.cp_peer_barrier(None, 0, 2, 1, 0, None) == I.CP_ERR_INVALID_ARG
+    assert lib.cp_peer_barrier(pads, 0, 17, 1, 0, None) == I.CP_ERR_UNSUPPORTED
+    assert lib.cp_peer_barrier((vp * 2)(1 << 20, None), 0, 2, 1, 0, None) == I.CP_ERR_INVALID_ARG
+    assert lib.cp_peer_barrier((vp * 2)(1 << 20, (2 << 20) + 2), 0, 2, 1, 0, None) == I.CP_ERR_MISALIGNED
 
     fetch = lib.cp_ring_fetch_block
     assert fetch(vp(1 << 20), vp(2 << 20), 1, 5, 2, 8, 4, 0, 8, 0, 2, None) == I.CP_ERR_INVALID_ARG  # past dst
