@@ -69,6 +69,18 @@ def mesh_coord(rank: int, ulysses_degree: int, ring_degree: int) -> MeshCoord:
     return MeshCoord(rank, u, g, tuple(g * U + j for j in range(U)), tuple(c * U + u for c in range(R)))
 
 
+def mesh_groups(coord: MeshCoord, group=None):
+    """This rank's Ulysses and ring process groups (for host barriers and exchanges).
+
+    Only the members of a group create it (``use_local_synchronization``), so every rank
+    makes two calls, and a group of some of the world's ranks works as well as the world.
+    """
+    ranks = dist.get_process_group_ranks(group) if group is not None else list(range(dist.get_world_size()))
+    ulysses = dist.new_group([ranks[r] for r in coord.ulysses_ranks], use_local_synchronization=True)
+    ring = dist.new_group([ranks[r] for r in coord.ring_ranks], use_local_synchronization=True)
+    return ulysses, ring
+
+
 def ring_order(ring_index: int, ring_degree: int) -> List[int]:
     """Blocks in the order a ring rank sees them: its own, then the block of the rank
     before it, and so on (K/V pass from rank i to rank i+1, "Ring Attention")."""
@@ -212,17 +224,8 @@ class ContextParallel:
         self.barrier_timeout_ms = int(barrier_timeout_ms)
         self.monitor = monitor
         self.device = torch.device("cuda", torch.cuda.current_device())
-        # Sub-groups for the host barrier: every rank creates every group, in one order.
-        self._pg = {"world": group, "ulysses": None, "ring": None}
-        ranks = dist.get_process_group_ranks(group) if group is not None else list(range(self.world))
-        for g in range(self.R):
-            pg = dist.new_group([ranks[g * self.U + j] for j in range(self.U)])
-            if g == self.coord.ring_index:
-                self._pg["ulysses"] = pg
-        for u in range(self.U):
-            pg = dist.new_group([ranks[c * self.U + u] for c in range(self.R)])
-            if u == self.coord.ulysses_index:
-                self._pg["ring"] = pg
+        ulysses, ring = mesh_groups(self.coord, group)
+        self._pg = {"world": group, "ulysses": ulysses, "ring": ring}
         self._epoch = {g: 0 for g in _GROUPS}
         self._pads = _PeerBuffer(_PAD_BYTES, self.rank, group)
         self._bufs: Dict[str, _PeerBuffer] = {}

@@ -16,7 +16,7 @@ import torch.multiprocessing as mp
 
 from context_attention_dit_b200 import binding
 from context_attention_dit_b200.distributed import (ContextParallel, HealthMonitor, PeerFailure, block_bounds,
-                                                    mesh_coord, ring_order)
+                                                    mesh_coord, mesh_groups, ring_order)
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -195,3 +195,41 @@ def test_rank_that_never_arrives_is_named_within_the_limit():
 def test_every_rank_arriving_passes():
     res, codes = _spawn(_failure_worker, 3, "all_arrive")
     assert codes == [0, 0, 0] and all(r == "ok" for r in res.values())
+
+
+def _groups_worker(rank, world, port, out, U, R, sub):
+    _init(rank, world, port)
+    import torch
+
+    # With `sub`, the mesh lives on the odd ranks only: the even ranks take no part.
+    group_ranks = list(range(1, world, 2)) if sub else list(range(world))
+    res = None
+    if rank in group_ranks:
+        group = dist.new_group(group_ranks, use_local_synchronization=True) if sub else None
+        me = dist.get_rank(group)
+        c = mesh_coord(me, U, R)
+        ulysses, ring = mesh_groups(c, group)
+        # Sum of the global ranks in each group: shows who is in it.
+        su = torch.tensor([rank])
+        dist.all_reduce(su, group=ulysses)
+        sr = torch.tensor([rank])
+        dist.all_reduce(sr, group=ring)
+        res = (me, int(su), int(sr))
+    out.put((rank, res))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("U,R,world,sub", [(2, 2, 4, False), (4, 1, 4, False), (1, 3, 3, False), (2, 2, 8, True)])
+def test_mesh_groups_hold_the_right_ranks(U, R, world, sub):
+    res, codes = _spawn(_groups_worker, world, U, R, sub)
+    assert codes == [0] * world
+    group_ranks = list(range(1, world, 2)) if sub else list(range(world))
+    for rank, r in res.items():
+        if rank not in group_ranks:
+            assert r is None
+            continue
+        me, su, sr = r
+        c = mesh_coord(me, U, R)
+        assert su == sum(group_ranks[x] for x in c.ulysses_ranks)
+        assert sr == sum(group_ranks[x] for x in c.ring_ranks)
