@@ -157,6 +157,12 @@ class HealthMonitor:
             missing = [r for r, k in enumerate(keys) if not self.store.check([k])]
             self.check()
             raise PeerFailure(missing, f"did not reach step {step} within {limit.total_seconds()} s") from e
+        # Every rank has set its key of this step, so every rank is done waiting on the
+        # previous one: this rank's key of that step can go (the store stays small).
+        try:
+            self.store.delete_key(self._key("step", step - 1, self.rank))
+        except Exception:
+            pass
 
 
 # ------------------------------------------------------------------ peer buffers
@@ -199,7 +205,7 @@ class ContextParallel:
     """Ulysses x ring attention over the ranks of a process group, one GPU per rank.
 
     Every rank calls the constructor and every method in the same order (the buffers are
-    allocated collectively).  ``barrier="device"`` orders steps with ``cp_peer_barrier``
+    allocated collectively), with its own GPU already current (``torch.cuda.set_device``).  ``barrier="device"`` orders steps with ``cp_peer_barrier``
     (stream-ordered, no host sync), whose wait gives up after ``barrier_timeout_ms``: ranks
     are driven by their hosts, so the limit must cover the host-side skew between ranks.
     A barrier that gave up leaves the step's outputs undefined; :meth:`check_device`

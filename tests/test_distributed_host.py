@@ -172,7 +172,12 @@ def _failure_worker(rank, world, port, out, mode):
         mon.arrive(1)
         mon.arrive(2)
         mon.check()
-        res = "ok"
+        dist.barrier()
+        # Step 1's keys are gone once every rank passed step 2; step 2's stay.
+        store = dist.distributed_c10d._get_default_store()
+        gone = not any(store.check([f"t{mode}/step/1/{r}"]) for r in range(world))
+        kept = all(store.check([f"t{mode}/step/2/{r}"]) for r in range(world))
+        res = "ok" if gone and kept else f"keys: step 1 gone {gone}, step 2 kept {kept}"
     out.put((rank, res))
     dist.barrier()
     dist.destroy_process_group()
@@ -194,7 +199,7 @@ def test_rank_that_never_arrives_is_named_within_the_limit():
 
 def test_every_rank_arriving_passes():
     res, codes = _spawn(_failure_worker, 3, "all_arrive")
-    assert codes == [0, 0, 0] and all(r == "ok" for r in res.values())
+    assert codes == [0, 0, 0] and all(r == "ok" for r in res.values()), res
 
 
 def _groups_worker(rank, world, port, out, U, R, sub):
