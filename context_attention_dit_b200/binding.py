@@ -42,7 +42,7 @@ EXPORTS = (
     "cp_debug_set_fault", "cp_last_device_status", "cp_status_string", "cp_version", "cp_usp_sim_workspace_size",
     "cp_usp_sim", "cp_ulysses_anything_permute", "cp_attn_merge_ulysses", "cp_peer_alloc", "cp_peer_open",
     "cp_peer_close", "cp_peer_free", "cp_ulysses_push_n", "cp_peer_barrier", "cp_ring_fetch_block",
-    "cp_ulysses_anything_push_n", "cp_attn_merge_push",
+    "cp_ulysses_anything_push_n", "cp_attn_merge_push", "cp_ulysses_anything_permute_n",
 )
 CP_PEER_MAX = 16
 CP_IPC_HANDLE_BYTES = 64
@@ -81,6 +81,9 @@ def load() -> ctypes.CDLL:
     lib.cp_ring_sim_static.argtypes = [vp, vp, vp, ip, i, vp, vp, i, i, i, i, i, f, i, vp]
     lib.cp_ulysses_permute.argtypes = [vp, vp, i, i, i, i, i, i, i, vp]
     lib.cp_ulysses_anything_permute.argtypes = [vp, vp, i, ip, ip, i, i, i, i, i, i, vp]
+    lib.cp_ulysses_anything_permute_n.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), i, i, ip, ip, i, i, i, i, i,
+                                                  i, vp]
+    lib.cp_ulysses_anything_permute_n.restype = ctypes.c_int
     lib.cp_ulysses_permute_n.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), i, i, i, i, i, i, i, i, vp]
     lib.cp_ulysses_permute_n.restype = ctypes.c_int
     lib.cp_ring_bounds.argtypes = [i, i, i, ip]
@@ -458,6 +461,33 @@ def ulysses_anything_permute(src, degree: int, seq_bounds: Sequence[int], head_b
                                             src.element_size(), ctypes.c_void_p(_stream(src)))
     _check(st, "cp_ulysses_anything_permute")
     return dst.view(-1)
+
+
+def ulysses_anything_permute_n(srcs, degree: int, seq_bounds: Sequence[int], head_bounds: Sequence[int], B: int,
+                               S: int, H: int, D: int, direction: int, dsts=None):
+    """:func:`ulysses_anything_permute` of several same-shaped packed buffers (e.g. Q, K, V)
+    in one launch; returns the destination buffers."""
+    srcs = list(srcs)
+    if not srcs:
+        raise ValueError("need at least one tensor")
+    ref = srcs[0]
+    for t in srcs:
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or not t.is_contiguous() or t.dtype != ref.dtype \
+                or t.device != ref.device or t.numel() != B * S * H * D:
+            raise ValueError(f"sources must be contiguous CUDA tensors of B*S*H*D = {B * S * H * D} elements, "
+                             f"one dtype and device")
+    if len(seq_bounds) != degree + 1 or len(head_bounds) != degree + 1:
+        raise ValueError("seq_bounds and head_bounds need degree + 1 entries")
+    dsts = [torch.empty(ref.numel(), dtype=ref.dtype, device=ref.device) for _ in srcs] if dsts is None else list(dsts)
+    n = len(srcs)
+    sp = (ctypes.c_void_p * n)(*[t.data_ptr() for t in srcs])
+    dp = (ctypes.c_void_p * n)(*[t.data_ptr() for t in dsts])
+    sb = (ctypes.c_int * (degree + 1))(*[int(x) for x in seq_bounds])
+    hb = (ctypes.c_int * (degree + 1))(*[int(x) for x in head_bounds])
+    st = load().cp_ulysses_anything_permute_n(sp, dp, n, degree, sb, hb, B, S, H, D, direction, ref.element_size(),
+                                              ctypes.c_void_p(_stream(ref)))
+    _check(st, "cp_ulysses_anything_permute_n")
+    return [d.view(-1) for d in dsts]
 
 
 def ring_bounds(S: int, n: int, anything: bool = False):

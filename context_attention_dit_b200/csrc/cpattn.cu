@@ -520,26 +520,41 @@ cp_status cp_attn_merge_ulysses(const float* partials, const float* lses, int n_
                       static_cast<cudaStream_t>(stream), degree, B);
 }
 
-cp_status cp_ulysses_anything_permute(const void* src, void* dst, int degree, const int* seq_bounds,
-                                      const int* head_bounds, int B, int S, int H, int D, int direction, int elem_bytes,
-                                      void* stream) {
-  NvtxRange nvtx_range("cp_ulysses_anything_permute");
+cp_status cp_ulysses_anything_permute_n(const void* const* srcs, void* const* dsts, int n_tensors, int degree,
+                                        const int* seq_bounds, const int* head_bounds, int B, int S, int H, int D,
+                                        int direction, int elem_bytes, void* stream) {
+  NvtxRange nvtx_range("cp_ulysses_anything_permute_n");
   if (degree < 1 || B < 0 || S < 0 || H < 0 || D < 0 || !seq_bounds || !head_bounds) return CP_ERR_INVALID_ARG;
   if (degree > kPermuteMaxDegree) return CP_ERR_UNSUPPORTED;
   if (direction != 0 && direction != 1) return CP_ERR_INVALID_ARG;
   if (elem_bytes != 2 && elem_bytes != 4) return CP_ERR_UNSUPPORTED;
+  if (n_tensors < 1 || !srcs || !dsts) return CP_ERR_INVALID_ARG;
+  if (n_tensors > kPermuteMaxTensors) return CP_ERR_UNSUPPORTED;
   if (seq_bounds[0] != 0 || seq_bounds[degree] != S || head_bounds[0] != 0 || head_bounds[degree] != H)
     return CP_ERR_INVALID_ARG;
   for (int i = 0; i < degree; ++i)
     if (seq_bounds[i] > seq_bounds[i + 1] || head_bounds[i] > head_bounds[i + 1]) return CP_ERR_INVALID_ARG;
   if (B == 0 || S == 0 || H == 0 || D == 0) return CP_OK;
-  if (!src || !dst) return CP_ERR_INVALID_ARG;
-  if (!aligned16(src) || !aligned16(dst)) return CP_ERR_MISALIGNED;
+  PermuteArgs a;
+  std::memset(&a, 0, sizeof(a));
+  for (int t = 0; t < n_tensors; ++t) {
+    if (!srcs[t] || !dsts[t]) return CP_ERR_INVALID_ARG;
+    if (!aligned16(srcs[t]) || !aligned16(dsts[t])) return CP_ERR_MISALIGNED;
+    a.src[t] = srcs[t];
+    a.dst[t] = dsts[t];
+  }
+  // No destination may overlap any source or another destination.
   const long long total = static_cast<long long>(B) * S * H * D * elem_bytes;
-  const char* s0 = static_cast<const char*>(src);
-  const char* d0 = static_cast<const char*>(dst);
-  if (s0 < d0 + total && d0 < s0 + total) return CP_ERR_INVALID_ARG;
-  if (static_cast<long long>(degree) * B > 65535 || static_cast<long long>(H) * D >= (1LL << 31))
+  for (int t = 0; t < n_tensors; ++t) {
+    const char* d0 = static_cast<const char*>(dsts[t]);
+    for (int u = 0; u < n_tensors; ++u) {
+      const char* s0 = static_cast<const char*>(srcs[u]);
+      if (s0 < d0 + total && d0 < s0 + total) return CP_ERR_INVALID_ARG;
+      const char* e0 = static_cast<const char*>(dsts[u]);
+      if (u != t && e0 < d0 + total && d0 < e0 + total) return CP_ERR_INVALID_ARG;
+    }
+  }
+  if (static_cast<long long>(n_tensors) * degree * B > 65535 || static_cast<long long>(H) * D >= (1LL << 31))
     return CP_ERR_UNSUPPORTED;
   DeviceInfo* dev = nullptr;
   cp_status st = device_info(&dev);
@@ -560,9 +575,8 @@ cp_status cp_ulysses_anything_permute(const void* src, void* dst, int degree, co
     using V = decltype(tag);
     const int ve = static_cast<int>(sizeof(V)) / elem_bytes;
     const int row_vecs = H * D / ve;
-    const dim3 grid((row_vecs + kPermuteThreads - 1) / kPermuteThreads, gy, degree * B);
-    ulysses_anything_kernel<V><<<grid, kPermuteThreads, 0, cs>>>(static_cast<const V*>(src), static_cast<V*>(dst), bd,
-                                                                 degree, B, S, H, D, ve, direction);
+    const dim3 grid((row_vecs + kPermuteThreads - 1) / kPermuteThreads, gy, n_tensors * degree * B);
+    ulysses_anything_kernel<V><<<grid, kPermuteThreads, 0, cs>>>(a, bd, degree, B, S, H, D, ve, direction);
   };
   if (row_bytes % 16 == 0)
     launch(uint4{});
@@ -573,6 +587,15 @@ cp_status cp_ulysses_anything_permute(const void* src, void* dst, int degree, co
   else
     launch(uint16_t{});
   return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+}
+
+cp_status cp_ulysses_anything_permute(const void* src, void* dst, int degree, const int* seq_bounds,
+                                      const int* head_bounds, int B, int S, int H, int D, int direction, int elem_bytes,
+                                      void* stream) {
+  NvtxRange nvtx_range("cp_ulysses_anything_permute");
+  // Pointers are checked by the batched form; nulls with empty sizes stay a no-op.
+  return cp_ulysses_anything_permute_n(&src, &dst, 1, degree, seq_bounds, head_bounds, B, S, H, D, direction,
+                                       elem_bytes, stream);
 }
 
 cp_status cp_ulysses_permute(const void* src, void* dst, int degree, int B, int S, int H, int D, int direction,

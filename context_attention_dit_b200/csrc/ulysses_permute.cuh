@@ -82,17 +82,21 @@ struct AnyBounds {
 
 // Walks the sequence-sharded rows: grid.x covers the vectors of a token row (VE elements
 // each, D a multiple of VE so no vector crosses a head), grid.y groups of kPermuteRows rows
-// of a shard (strided by gridDim.y), grid.z = p * B + b.  Each thread finds the head group
-// of its vector once and reuses it for every row.
+// of a shard (strided by gridDim.y), grid.z = (tensor * P + p) * B + b.  Each thread finds
+// the head group of its vector once and reuses it for every row.
 template <typename V>
 __global__ void __launch_bounds__(kPermuteThreads)
-    ulysses_anything_kernel(const V* __restrict__ src, V* __restrict__ dst, const __grid_constant__ AnyBounds bd,
-                            int P, int B, int S, int H, int D, int VE, int direction) {
+    ulysses_anything_kernel(const __grid_constant__ PermuteArgs a, const __grid_constant__ AnyBounds bd, int P, int B,
+                            int S, int H, int D, int VE, int direction) {
   const int row_vecs = H * D / VE;
   const int i = blockIdx.x * kPermuteThreads + threadIdx.x;
   if (i >= row_vecs) return;
-  const int p = blockIdx.z / B;
-  const int b = blockIdx.z - p * B;
+  const int n = blockIdx.z / (P * B);
+  const int pb = blockIdx.z - n * (P * B);
+  const int p = pb / B;
+  const int b = pb - p * B;
+  const V* __restrict__ src = static_cast<const V*>(a.src[n]);
+  V* __restrict__ dst = static_cast<V*>(a.dst[n]);
   const int s0 = bd.seq[p];
   const int Sp = bd.seq[p + 1] - s0;
   const long long e = static_cast<long long>(i) * VE;  // element within the token row

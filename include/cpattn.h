@@ -263,6 +263,18 @@ CP_API cp_status cp_ulysses_anything_permute(const void* src, void* dst, int deg
                                              int elem_bytes, void* stream);
 
 /*
+ * cp_ulysses_anything_permute_n - cp_ulysses_anything_permute of n_tensors same-shaped
+ * tensors in one launch (Q, K and V move together).
+ *
+ * srcs, dsts: HOST arrays of n_tensors device pointers (1 <= n_tensors <= 8), read during
+ * the call only.  Other arguments and rules as cp_ulysses_anything_permute; no destination
+ * may overlap any source or another destination (CP_ERR_INVALID_ARG).
+ */
+CP_API cp_status cp_ulysses_anything_permute_n(const void* const* srcs, void* const* dsts, int n_tensors, int degree,
+                                               const int* seq_bounds, const int* head_bounds, int B, int S, int H,
+                                               int D, int direction, int elem_bytes, void* stream);
+
+/*
  * cp_ulysses_permute - the Ulysses all-to-all, simulated as one local copy.
  *
  * Source: "Context parallelism", "Ulysses Attention" and the variants table

@@ -309,3 +309,19 @@ def test_merge_push_checks_before_cuda(lib):
     assert call(vp(1 << 20), (vp * 2)(3 << 20, (4 << 20) + 8), 0, 2, 8, 4) == I.CP_ERR_MISALIGNED
     assert call(vp(1 << 20), (vp * 2)(3 << 20, None), 0, 2, 8, 4) == I.CP_ERR_INVALID_ARG
     assert call(None, None, 0, 2, 0, 4) == I.CP_OK  # empty
+
+
+def test_anything_permute_n_checks_before_cuda(lib):
+    vp = ctypes.c_void_p
+    sb, hb = _bounds(0, 3, 5), _bounds(0, 2, 3)
+    srcs, dsts = (vp * 2)(1 << 20, 2 << 20), (vp * 2)(3 << 20, 4 << 20)
+    call = lambda s, d, n, sbd=sb, hbd=hb, S=5, H=3: lib.cp_ulysses_anything_permute_n(  # noqa: E731
+        s, d, n, 2, sbd, hbd, 1, S, H, 8, 0, 2, None)
+    assert call(srcs, dsts, 0) == I.CP_ERR_INVALID_ARG
+    assert call(srcs, dsts, 9) == I.CP_ERR_UNSUPPORTED
+    assert call(srcs, dsts, 2, S=6) == I.CP_ERR_INVALID_ARG  # seq bounds must end at S
+    assert call(srcs, (vp * 2)(3 << 20, 3 << 20), 2) == I.CP_ERR_INVALID_ARG  # destinations overlap
+    assert call(srcs, (vp * 2)(3 << 20, 1 << 20), 2) == I.CP_ERR_INVALID_ARG  # a destination on a source
+    assert call(srcs, (vp * 2)(3 << 20, (4 << 20) + 8), 2) == I.CP_ERR_MISALIGNED
+    assert call(srcs, (vp * 2)(3 << 20, None), 2) == I.CP_ERR_INVALID_ARG
+    assert call(srcs, dsts, 2, S=0, sbd=_bounds(0, 0, 0)) == I.CP_OK  # empty

@@ -53,6 +53,23 @@ def test_anything_bit_exact(case):
     assert torch.equal(back.cpu(), pack_seq(x, sb))
 
 
+@pytest.mark.parametrize("case", [CASES[0], CASES[2], CASES[3]], ids=["flux1008_p4", "empty_heads", "empty_seq"])
+def test_anything_batched_bit_exact(case):
+    """Q, K and V in one launch: each equals the oracle's exchange of that tensor."""
+    P, B, S, H, D, dtype, sb, hb = case
+    sb = sb or near_even(S, P)
+    hb = hb or near_even(H, P)
+    g = torch.Generator().manual_seed(S * 17 + H)
+    xs = [torch.randn(B, S, H, D, generator=g).to(dtype) for _ in range(3)]
+    ys = binding.ulysses_anything_permute_n([pack_seq(x, sb).cuda() for x in xs], P, sb, hb, B, S, H, D, 0)
+    for x, y in zip(xs, ys):
+        ref = oracle.ulysses_anything_fwd([x[:, sb[p]:sb[p + 1]] for p in range(P)], sb, hb)
+        assert torch.equal(y.cpu(), torch.cat([r.reshape(-1) for r in ref]))
+    backs = binding.ulysses_anything_permute_n(ys, P, sb, hb, B, S, H, D, 1)
+    for x, b in zip(xs, backs):
+        assert torch.equal(b.cpu(), pack_seq(x, sb))
+
+
 def test_anything_equals_even_exchange_on_equal_shards():
     P, B, S, H, D = 8, 1, 4608, 24, 128
     x = torch.randn(P, B, S // P, H, D, generator=torch.Generator().manual_seed(3)).bfloat16().cuda()
