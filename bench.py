@@ -594,6 +594,11 @@ def run_profile_case(args):
             xs = [t.view(B, P, S // P, H, D).permute(1, 0, 2, 3, 4).contiguous() for t in (q, k, v)]
             ys = binding.ulysses_permute_n(xs, P, 0)
             binding.ulysses_permute(ys[0], P, 1)
+        elif case == "anything":  # Q/K/V Ulysses-Anything exchange, FLUX-1008^2 (4481 tokens) over 4
+            Sa = 4481
+            xa = [torch.randn(B * Sa * H * D, device="cuda").bfloat16() for _ in range(3)]
+            binding.ulysses_anything_permute_n(xa, 4, binding.ring_bounds(Sa, 4, anything=True),
+                                               binding.ring_bounds(H, 4, anything=True), B, Sa, H, D, 0)
         elif case == "push":  # every rank's Q/K/V push, ranks by turns, local buffers for the peers'
             xs = [t.view(B, P, S // P, H, D).permute(1, 0, 2, 3, 4).contiguous() for t in (q, k, v)]
             ys = [torch.empty(P, B, S, H // P, D, dtype=torch.bfloat16, device="cuda") for _ in range(3)]
@@ -615,7 +620,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-budget", type=float, default=90.0)
-    ap.add_argument("--profile-case", choices=["attn_ring1", "attn_ring8", "merge", "permute", "push"], default=None)
+    ap.add_argument("--profile-case", choices=["attn_ring1", "attn_ring8", "merge", "permute", "push", "anything"], default=None)
     ap.add_argument("--profile-batch", type=int, default=2)
     ap.add_argument("--profile-reps", type=int, default=3)
     args = ap.parse_args()
