@@ -1,4 +1,4 @@
-"""ContextParallel with real processes: 2 to 4 ranks, each its own process and CUDA
+"""ContextParallel with real processes: 2 to 8 ranks, each its own process and CUDA
 context, sharing the one GPU of the test box through CUDA IPC.
 
 The peer buffers, the pushes into other processes' memory, the copy-engine fetches and
@@ -128,6 +128,9 @@ def _run(U, R, B, H, D, lens, oracle_check=False):
         (1, 2, 2, 3, 128, [301, 300], True),  # ring anything: uneven blocks
         (1, 3, 1, 2, 64, [384, 384, 384], False),  # ring of three
         (2, 2, 1, 4, 64, [256, 256, 256, 256], True),  # unified: 2 x 2 mesh
+        (8, 1, 1, 24, 128, [576] * 8, False),  # Ulysses-8 on the FLUX-like shape: eight processes
+        (4, 2, 1, 8, 128, [128] * 8, False),  # unified 4 x 2
+        (2, 4, 1, 4, 64, [96] * 8, False),  # unified 2 x 4
     ],
 )
 def test_context_parallel_matches_single_process(U, R, B, H, D, lens, oracle_check):
