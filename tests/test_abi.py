@@ -325,3 +325,20 @@ def test_anything_permute_n_checks_before_cuda(lib):
     assert call(srcs, (vp * 2)(3 << 20, (4 << 20) + 8), 2) == I.CP_ERR_MISALIGNED
     assert call(srcs, (vp * 2)(3 << 20, None), 2) == I.CP_ERR_INVALID_ARG
     assert call(srcs, dsts, 2, S=0, sbd=_bounds(0, 0, 0)) == I.CP_OK  # empty
+
+
+def test_peer_bindings_reject_bad_arguments_before_the_library():
+    import torch
+
+    with pytest.raises(ValueError):
+        binding.peer_open(b"\0" * 10)  # an IPC handle has 64 bytes
+    with pytest.raises(ValueError):
+        binding.ulysses_push_n([1 << 20], [[2 << 20]], 0, 2, 1, 4, 4, 8, 0, 2, 0)  # one row of 1 != degree 2
+    with pytest.raises(ValueError):
+        binding.ulysses_push_n([1 << 20, 2 << 20], [[3 << 20, 4 << 20]], 0, 2, 1, 4, 4, 8, 0, 2, 0)  # rows != sources
+    with pytest.raises(ValueError):
+        binding.ulysses_anything_push_n([1 << 20], [[2 << 20, 3 << 20]], 0, [0, 2, 4], [0, 2], 1, 2, 8, 0, 2, 0)
+    with pytest.raises(ValueError):  # host tensors never reach the library
+        binding.attn_merge_push(torch.zeros(1, 1, 4, 1, 64), torch.zeros(1, 1, 1, 4), [1 << 20, 2 << 20], 0)
+    with pytest.raises(ValueError):
+        binding.ulysses_anything_permute_n([torch.zeros(8)], 2, [0, 1, 2], [0, 1, 2], 1, 2, 2, 2, 0)
