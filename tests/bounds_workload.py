@@ -52,6 +52,35 @@ def run():
         xa = torch.randn(2 * Sa * Ha * Da, generator=torch.Generator().manual_seed(7)).bfloat16().cuda()
         ya = binding.ulysses_anything_permute(xa, Pa, sb, hb, 2, Sa, Ha, Da, 0)
         record(f"anything_{Pa}_{Sa}_{Ha}_{Da}", ya, binding.ulysses_anything_permute(ya, Pa, sb, hb, 2, Sa, Ha, Da, 1))
+    yn = binding.ulysses_anything_permute_n([xa, xa.clone()], Pa, sb, hb, 2, Sa, Ha, Da, 0)
+    record("anything_n", *yn)
+    # One process per GPU, the ranks taken in turn with local buffers for their peers'.
+    st = torch.cuda.current_stream().cuda_stream
+    ys = [torch.zeros(B, S, H // P, D, dtype=torch.bfloat16, device="cuda") for _ in range(P)]
+    for r in range(P):
+        binding.ulysses_push_n([src[r].data_ptr()], [[t.data_ptr() for t in ys]], r, P, B, S, H, D, 0, 2, st)
+    xb = [torch.zeros(B, S // P, H, D, dtype=torch.bfloat16, device="cuda") for _ in range(P)]
+    for r in range(P):
+        binding.ulysses_push_n([ys[r].data_ptr()], [[t.data_ptr() for t in xb]], r, P, B, S, H, D, 1, 2, st)
+    record("push", *ys, *xb)
+    outs = [torch.zeros(B, S // P, H, D, dtype=torch.bfloat16, device="cuda") for _ in range(P)]
+    for u in range(P):
+        binding.attn_merge_push(parts[:, u * B:(u + 1) * B].contiguous(), lses[:, u * B:(u + 1) * B].contiguous(),
+                                [o.data_ptr() for o in outs], u)
+    record("merge_push", *outs)
+    xf = torch.randn(2, Sa, Ha, Da, generator=torch.Generator().manual_seed(9)).bfloat16().cuda()
+    xs = [xf[:, sb[p]:sb[p + 1]].contiguous() for p in range(Pa)]
+    ya = [torch.zeros(2, Sa, hb[q + 1] - hb[q], Da, dtype=torch.bfloat16, device="cuda") for q in range(Pa)]
+    xr = [torch.zeros(2, sb[p + 1] - sb[p], Ha, Da, dtype=torch.bfloat16, device="cuda") for p in range(Pa)]
+    ptr = lambda t: t.data_ptr() if t.numel() else 16  # noqa: E731  (an empty shard is never touched)
+    for r in range(Pa):
+        binding.ulysses_anything_push_n([ptr(xs[r])], [[ptr(t) for t in ya]], r, sb, hb, 2, Ha, Da, 0, 2, st)
+    for r in range(Pa):
+        binding.ulysses_anything_push_n([ptr(ya[r])], [[ptr(t) for t in xr]], r, sb, hb, 2, Ha, Da, 1, 2, st)
+    record("anything_push", *ya, *xr)
+    pad = torch.zeros(16, dtype=torch.int32, device="cuda")
+    binding.peer_barrier([pad.data_ptr()], 0, 1, st)
+    record("barrier", pad)
     shards = [t.reshape(1, 2, 128, 4, 128).permute(1, 0, 2, 3, 4).contiguous().cuda()
               for t in make_qkv(1, 4, 256, 256, 128, seed=8)]
     o, lse, _ = binding.usp_sim(*shards, 2, [0, 100, 256])
