@@ -104,6 +104,16 @@ def exchange(obj, group=None) -> list:
     return out
 
 
+def shard_shapes(shape, group=None) -> List[Tuple[int, int, int, int]]:
+    """Every rank's (B, S_local, H, D) shard shape, by rank (a host exchange).  Every rank
+    gets the same list, so a mismatch in batch, heads or head_dim raises on all ranks
+    alike, before anyone launches an exchange that could not complete."""
+    shapes = [tuple(int(x) for x in t) for t in exchange(tuple(int(x) for x in shape), group)]
+    if any(len(t) != 4 for t in shapes) or len({(b, h, d) for b, _, h, d in shapes}) != 1:
+        raise ValueError(f"ranks disagree on batch, heads or head_dim: {shapes}")
+    return shapes
+
+
 # ------------------------------------------------------------------ failure detection
 
 
@@ -305,12 +315,8 @@ class ContextParallel:
     # -- the step
 
     def shard_shapes(self, q) -> List[Tuple[int, int, int, int]]:
-        """Every rank's (B, S_local, H, D), by rank (a host exchange over the group).  All
-        ranks get the same list, so a mismatch raises on every rank alike."""
-        shapes = [tuple(int(x) for x in t) for t in exchange(tuple(q.shape), self.group)]
-        if len({(b, h, d) for b, _, h, d in shapes}) != 1:
-            raise ValueError(f"ranks disagree on batch, heads or head_dim: {shapes}")
-        return shapes
+        """Every rank's (B, S_local, H, D), by rank (see :func:`shard_shapes`)."""
+        return shard_shapes(tuple(q.shape), self.group)
 
     def attention(self, q, k, v, scale: Optional[float] = None,
                   seq_lengths: Optional[Sequence[int]] = None) -> torch.Tensor:

@@ -16,7 +16,7 @@ import torch.multiprocessing as mp
 
 from context_attention_dit_b200 import binding
 from context_attention_dit_b200.distributed import (ContextParallel, HealthMonitor, PeerFailure, block_bounds,
-                                                    mesh_coord, mesh_groups, ring_order)
+                                                    mesh_coord, mesh_groups, ring_order, shard_shapes)
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -238,3 +238,26 @@ def test_mesh_groups_hold_the_right_ranks(U, R, world, sub):
         c = mesh_coord(me, U, R)
         assert su == sum(group_ranks[x] for x in c.ulysses_ranks)
         assert sr == sum(group_ranks[x] for x in c.ring_ranks)
+
+
+def _shapes_worker(rank, world, port, out, mismatch):
+    _init(rank, world, port)
+    # Uneven sequence shards are fine; a rank with other heads is an error on every rank.
+    H = 8 if not (mismatch and rank == 1) else 6
+    try:
+        res = shard_shapes((1, 100 + rank, H, 128))
+    except ValueError as e:
+        res = "error: " + str(e)
+    out.put((rank, res))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_shard_shapes_are_shared_and_mismatches_raise_everywhere():
+    res, codes = _spawn(_shapes_worker, 3, False)
+    assert codes == [0, 0, 0]
+    for r in range(3):
+        assert res[r] == [(1, 100, 8, 128), (1, 101, 8, 128), (1, 102, 8, 128)]
+    res, codes = _spawn(_shapes_worker, 3, True)
+    assert codes == [0, 0, 0]
+    assert all(isinstance(v, str) and v.startswith("error: ranks disagree") for v in res.values())
