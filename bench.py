@@ -202,7 +202,15 @@ def run_ours(args):
     lse_full = torch.empty((B, H, S), dtype=torch.float32, device=dev)
     o_seq = torch.empty((P, B, S // P, H, D), dtype=torch.bfloat16, device=dev)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+    # L2 flush between timed steps: a read-only sweep of a buffer larger than L2.  A write
+    # would leave L2 full of dirty lines that the next kernel has to write back; a read
+    # evicts the previous step's dirty lines during the flush and leaves only clean ones.
+    flush_buf = torch.ones(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=dev)
+    flush_sink = torch.empty((), dtype=torch.float32, device=dev)
+    flush_mib = flush_buf.numel() * 4 >> 20
+
+    def flush_l2():
+        torch.sum(flush_buf, dtype=torch.float32, out=flush_sink)
     scale = w.scale
     flop = w.flop
     launches_per_step = 1 + 1 + 1  # exchange of Q, K, V; attention; merge fused with the inverse exchange
@@ -226,7 +234,7 @@ def run_ours(args):
             evs[3].record()
 
     for _ in range(args.warmup):
-        flush.zero_()
+        flush_l2()
         step()
     torch.cuda.synchronize()
     assert binding.last_device_status() == 0
@@ -239,7 +247,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     clocks.mark_start()
     for i in range(args.steps):
-        flush.zero_()
+        flush_l2()
         step(evs[i])
     torch.cuda.synchronize()
     clocks.mark_end()
@@ -260,7 +268,7 @@ def run_ours(args):
     l1 = torch.empty((B, H, S), dtype=torch.float32, device=dev)
     r1 = []
     for i in range(max(args.warmup, 3) + 50):
-        flush.zero_()
+        flush_l2()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         binding.attn_fwd(qd, kd, vd, scale=scale, out=o1, lse=l1)
@@ -276,7 +284,7 @@ def run_ours(args):
     view = lambda t: t.view(Bp, S, Hp, D)
     rf = []
     for i in range(max(args.warmup, 3) + 50):
-        flush.zero_()
+        flush_l2()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         binding.ring_sim_fused(view(yq), view(yk), view(yv), bounds, scale=scale, out=fo, out_lse=fl)
@@ -288,7 +296,7 @@ def run_ours(args):
     def timed_ms(fn, reps=20):
         evs = []
         for i in range(max(args.warmup, 3) + reps):
-            flush.zero_()
+            flush_l2()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
             fn()
@@ -296,6 +304,18 @@ def run_ours(args):
             evs.append((a, b))
         torch.cuda.synchronize()
         return statistics.mean(a.elapsed_time(b) for a, b in evs[max(args.warmup, 3):])
+
+    # The step in two launches: the exchange of Q/K/V, then the ring with the LSE merge
+    # carried in TMEM across the blocks and the inverse exchange in the kernel's epilogue
+    # (cp_ring_sim_fused_ulysses): no fp32 partials and no merge pass.
+    o_seq2 = torch.empty_like(o_seq)
+    lse2 = torch.empty_like(lse_full)
+
+    def step2():
+        binding.ulysses_permute_n((xq, xk, xv), P, 0, dsts=(yq, yk, yv))
+        binding.ring_sim_fused_ulysses(yq, yk, yv, P, bounds, scale=scale, out=o_seq2, out_lse=lse2)
+
+    step2_ms = timed_ms(step2, reps=50)
 
     # Unified SP: Ulysses 2 x ring 4 and Ulysses 4 x ring 2 on the same tensors, through
     # cp_usp_sim (exchange, ring attention + merge, inverse exchange, LSE regroup).
@@ -319,7 +339,12 @@ def run_ours(args):
     sba, hba = binding.ring_bounds(Sa, 4, anything=True), binding.ring_bounds(H, 4, anything=True)
     any_ms = timed_ms(lambda: binding.ulysses_anything_permute_n(xa, 4, sba, hba, B, Sa, H, D, 0, dsts=ya))
     any_bytes = 2 * sum(t.numel() * t.element_size() for t in xa)
-    del xa, ya
+    # Ring Anything's pad -> all-gather buffer of K and V for the same 4481 tokens over 4.
+    ka = [t.view(B, Sa, H, D) for t in xa[1:]]
+    ga = [torch.empty((4, B, 1121, H, D), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    gather_ms = timed_ms(lambda: binding.ring_anything_gather(ka, sba, 1121, dsts=ga))
+    gather_bytes = sum(t.numel() * t.element_size() for t in ka) + sum(t.numel() * t.element_size() for t in ga)
+    del xa, ya, ka, ga
 
     # The other workloads (parity cases, reported beside the bench line, not as it): ring /
     # ring-anything attention, blocks + LSE merge (cp_ring_sim), over each of their splits.
@@ -335,9 +360,12 @@ def run_ours(args):
             cl = torch.empty((wl.B, wl.H, wl.S), dtype=torch.float32, device=dev)
             ms = timed_ms(lambda: binding.ring_sim(cq, ck, cv, bnd, scale=wl.scale, workspace=cws, out=co,
                                                    out_lse=cl), reps=5 if wl.S > 20000 else 20)
+            fms = timed_ms(lambda: binding.ring_sim_fused(cq, ck, cv, bnd, scale=wl.scale, out=co, out_lse=cl),
+                           reps=5 if wl.S > 20000 else 20)
             key = name if len(wl.splits) == 1 else f"{name}_split{i}"
             other_configs[key] = {"blocks": list(sizes), "ms": round(ms, 4),
-                                  "tflops": round(wl.flop / (ms * 1e-3) / 1e12, 2)}
+                                  "tflops": round(wl.flop / (ms * 1e-3) / 1e12, 2),
+                                  "fused_ms": round(fms, 4), "fused_tflops": round(wl.flop / (fms * 1e-3) / 1e12, 2)}
             del cws, co, cl
         del cq, ck, cv
     torch.cuda.empty_cache()
@@ -416,6 +444,8 @@ def run_ours(args):
         merge_bytes = n_blocks * rows * (4 * D + 4) + rows * (2 * D + 4)
         perm_bytes = 3 * 2 * B * S * H * D * 2
         part_bytes = n_blocks * rows * (4 * D + 4)
+        merge_gbs = merge_bytes / (statistics.mean(merge_ms) * 1e-3) / 1e9
+        perm_gbs = perm_bytes / (statistics.mean(perm_ms) * 1e-3) / 1e9
         line = {
             "metric": METRIC,
             "value": round(value, 2),
@@ -431,7 +461,7 @@ def run_ours(args):
             "data": "synthetic (seeded N(0,1) bf16, per-head RMS-normed Q/K; sha256 " + ",".join(
                 f"{k}:{v}" for k, v in sha.items()) + ")",
             "config": step_config(world, B, S, H, D, P, n_blocks,
-                                  "flushed between timed steps (write of %d MiB > L2)" % (flush.numel() >> 20)),
+                                  "flushed between timed steps (read of %d MiB > L2)" % flush_mib),
             "roofline": {
                 "kernel": "attn_fwd_sm100 (8 ring blocks in one launch)",
                 "bound": "tensor",
@@ -454,11 +484,19 @@ def run_ours(args):
                 "ring8_fused_ms": round(fused_ms, 4),
                 "ring8_fused_tflops": round(flop / (fused_ms * 1e-3) / 1e12, 2),
                 "attn_ring8_partial_bytes": part_bytes,
+                "step_2launch_fused_ulysses_ms": round(step2_ms, 4),
+                "step_2launch_fused_ulysses_tflops": round(flop / (step2_ms * 1e-3) / 1e12, 2),
                 "merge_inverse_exchange_ms": round(statistics.mean(merge_ms), 4),
-                "merge_inverse_exchange_gbs": round(merge_bytes / (statistics.mean(merge_ms) * 1e-3) / 1e9, 1),
+                "merge_inverse_exchange_gbs": round(merge_gbs, 1),
+                "merge_inverse_exchange_frac_of_measured_hbm": round(merge_gbs / peaks["hbm_gbs"], 4),
+                "merge_inverse_exchange_frac_of_spec_8000": round(merge_gbs / 8000.0, 4),
                 "permute_qkv_ms": round(statistics.mean(perm_ms), 4),
-                "permute_qkv_gbs": round(perm_bytes / (statistics.mean(perm_ms) * 1e-3) / 1e9, 1),
+                "permute_qkv_gbs": round(perm_gbs, 1),
+                "permute_qkv_frac_of_measured_hbm": round(perm_gbs / peaks["hbm_gbs"], 4),
+                "permute_qkv_frac_of_spec_8000": round(perm_gbs / 8000.0, 4),
                 "hbm_peak_gbs": peaks["hbm_gbs"],
+                "ring_anything_gather_kv_flux1008_r4_ms": round(gather_ms, 4),
+                "ring_anything_gather_kv_flux1008_r4_gbs": round(gather_bytes / (gather_ms * 1e-3) / 1e9, 1),
                 **usp,
                 "anything_permute_qkv_flux1008_p4_ms": round(any_ms, 4),
                 "anything_permute_qkv_flux1008_p4_gbs": round(any_bytes / (any_ms * 1e-3) / 1e9, 1),
@@ -598,6 +636,10 @@ def run_profile_case(args):
             xa = [torch.randn(B * Sa * H * D, device="cuda").bfloat16() for _ in range(3)]
             binding.ulysses_anything_permute_n(xa, 4, binding.ring_bounds(Sa, 4, anything=True),
                                                binding.ring_bounds(H, 4, anything=True), B, Sa, H, D, 0)
+        elif case == "gather":  # Ring Anything pad -> all-gather buffer of K/V, FLUX-1008^2 over 4
+            Sa = 4481
+            ka = [torch.randn(B, Sa, H, D, device="cuda").bfloat16() for _ in range(2)]
+            binding.ring_anything_gather(ka, binding.ring_bounds(Sa, 4, anything=True))
         elif case == "push":  # every rank's Q/K/V push, ranks by turns, local buffers for the peers'
             xs = [t.view(B, P, S // P, H, D).permute(1, 0, 2, 3, 4).contiguous() for t in (q, k, v)]
             ys = [torch.empty(P, B, S, H // P, D, dtype=torch.bfloat16, device="cuda") for _ in range(3)]
@@ -619,7 +661,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-budget", type=float, default=90.0)
-    ap.add_argument("--profile-case", choices=["attn_ring1", "attn_ring8", "merge", "permute", "push", "anything"], default=None)
+    ap.add_argument("--profile-case", choices=["attn_ring1", "attn_ring8", "merge", "permute", "push", "anything", "gather"], default=None)
     ap.add_argument("--profile-batch", type=int, default=2)
     ap.add_argument("--profile-reps", type=int, default=3)
     args = ap.parse_args()

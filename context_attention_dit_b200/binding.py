@@ -42,7 +42,8 @@ EXPORTS = (
     "cp_debug_set_fault", "cp_last_device_status", "cp_status_string", "cp_version", "cp_usp_sim_workspace_size",
     "cp_usp_sim", "cp_ulysses_anything_permute", "cp_attn_merge_ulysses", "cp_peer_alloc", "cp_peer_open",
     "cp_peer_close", "cp_peer_free", "cp_ulysses_push_n", "cp_peer_barrier", "cp_ring_fetch_block",
-    "cp_ulysses_anything_push_n", "cp_attn_merge_push", "cp_ulysses_anything_permute_n",
+    "cp_ulysses_anything_push_n", "cp_attn_merge_push", "cp_ulysses_anything_permute_n", "cp_attn_fwd_strided",
+    "cp_ring_sim_fused_ulysses", "cp_ring_anything_gather",
 )
 CP_PEER_MAX = 16
 CP_IPC_HANDLE_BYTES = 64
@@ -67,6 +68,13 @@ def load() -> ctypes.CDLL:
     vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     ip = ctypes.POINTER(ctypes.c_int)
     lib.cp_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
+    ll = ctypes.c_longlong
+    lib.cp_attn_fwd_strided.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, ll, ll, ll, ll, ll, ll, f, i, vp]
+    lib.cp_attn_fwd_strided.restype = ctypes.c_int
+    lib.cp_ring_sim_fused_ulysses.argtypes = [vp, vp, vp, i, ip, i, vp, vp, i, i, i, i, f, i, vp]
+    lib.cp_ring_sim_fused_ulysses.restype = ctypes.c_int
+    lib.cp_ring_anything_gather.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), i, ip, i, i, i, i, i, i, i, vp]
+    lib.cp_ring_anything_gather.restype = ctypes.c_int
     lib.cp_attn_fwd_blocks.argtypes = [vp, vp, vp, ip, i, vp, vp, i, i, i, i, i, f, vp]
     lib.cp_attn_merge.argtypes = [vp, vp, i, vp, vp, i, i, i, i, i, vp]
     lib.cp_attn_merge_ulysses.argtypes = [vp, vp, i, vp, vp, i, i, i, i, i, i, vp]
@@ -169,6 +177,51 @@ def attn_fwd(q, k, v, scale: Optional[float] = None, out_dtype=torch.bfloat16, o
     st = load().cp_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Sq, Skv, D, scale, code,
                             ctypes.c_void_p(_stream(q)))
     _check(st, "cp_attn_fwd")
+    return out, lse
+
+
+def _check_view(name: str, t, D: Optional[int] = None):
+    """A 4-D bf16 CUDA view whose heads and head_dim are dense (strides (., ., D, 1))."""
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dim() != 4:
+        raise ValueError(f"{name} must be 4-D (batch, seq, heads, head_dim), got {tuple(t.shape)}")
+    d = t.shape[3]
+    if t.stride(3) != 1 or (t.shape[2] > 1 and t.stride(2) != d):
+        raise ValueError(f"{name}: heads and head_dim must be dense (strides (., ., {d}, 1)), got {t.stride()}")
+    return t.stride(0), t.stride(1)
+
+
+def attn_fwd_strided(q, k, v, scale: Optional[float] = None, out_dtype=torch.bfloat16, out=None, lse=None,
+                     want_lse: bool = True):
+    """:func:`attn_fwd` on views: q, k, v (and ``out`` if given) may be slices of larger
+    tensors along batch and sequence (e.g. ``k_full[:, c0:c1]``), with heads and head_dim
+    dense.  Returns ``(out, lse)``; ``lse`` is dense ``[B, H, Sq]``."""
+    for name, t in (("query", q), ("key", k), ("value", v)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16:
+            raise ValueError(f"{name} must be a bfloat16 tensor")
+    q_sb, q_ss = _check_view("query", q)
+    kv_sb, kv_ss = _check_view("key", k)
+    if _check_view("value", v) != (kv_sb, kv_ss):
+        raise ValueError("key and value must have the same strides")
+    if not (q.device == k.device == v.device):
+        raise ValueError("query, key and value must be on the same device")
+    B, Sq, H, D = q.shape
+    Skv = k.shape[1]
+    if k.shape != v.shape or k.shape[0] != B or k.shape[2] != H or k.shape[3] != D:
+        raise ValueError(f"incompatible shapes q{tuple(q.shape)} k{tuple(k.shape)} v{tuple(v.shape)}")
+    code = _out_code(out_dtype)
+    scale = float(D ** -0.5 if scale is None else scale)
+    if out is None:
+        out = torch.empty((B, Sq, H, D), dtype=out_dtype, device=q.device)
+    if out.dtype != out_dtype or tuple(out.shape) != (B, Sq, H, D) or out.device != q.device:
+        raise ValueError(f"out must be {out_dtype} of shape {(B, Sq, H, D)} on {q.device}")
+    o_sb, o_ss = _check_view("out", out)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
+    st = load().cp_attn_fwd_strided(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Sq, Skv, D, q_sb, q_ss,
+                                    kv_sb, kv_ss, o_sb, o_ss, scale, code, ctypes.c_void_p(_stream(q)))
+    _check(st, "cp_attn_fwd_strided")
     return out, lse
 
 
@@ -327,6 +380,75 @@ def ring_sim_fused(q, k, v, chunk_bounds: Sequence[int], scale: Optional[float] 
                                   scale, code, ctypes.c_void_p(_stream(q)))
     _check(st, "cp_ring_sim_fused")
     return out, out_lse
+
+
+def ring_sim_fused_ulysses(q, k, v, degree: int, chunk_bounds: Sequence[int], scale: Optional[float] = None,
+                           out_dtype=torch.bfloat16, out=None, out_lse=None):
+    """Fused ring attention on Ulysses head shards writing the token-sharded output.
+
+    q, k, v: head-sharded ``[degree, B, S, H/degree, D]`` bf16 (the output of
+    :func:`ulysses_permute` direction 0).  Returns ``(out [degree, B, S/degree, H, D],
+    lse [B, H, S])``: what :func:`usp_sim` returns for the same sequence-sharded inputs.
+    """
+    for name, t in (("query", q), ("key", k), ("value", v)):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.bfloat16 or t.dim() != 5:
+            raise ValueError(f"{name} must be a 5-D bf16 CUDA tensor [degree, B, S, H/degree, D]")
+        if not t.is_contiguous() or t.shape != q.shape or t.device != q.device:
+            raise ValueError("query, key and value must be contiguous, of one shape, on one device")
+    P, B, S, Hp, D = q.shape
+    if P != degree:
+        raise ValueError(f"leading dimension {P} != degree {degree}")
+    if S % P:
+        raise ValueError(f"sequence {S} not divisible by degree {P}")
+    H = Hp * P
+    code = _out_code(out_dtype)
+    scale = float(D ** -0.5 if scale is None else scale)
+    n = len(chunk_bounds) - 1
+    if n < 1:
+        raise ValueError("chunk_bounds needs at least two entries")
+    bounds = (ctypes.c_int * (n + 1))(*[int(c) for c in chunk_bounds])
+    if out is None:
+        out = torch.empty((P, B, S // P, H, D), dtype=out_dtype, device=q.device)
+    if out_lse is None:
+        out_lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    st = load().cp_ring_sim_fused_ulysses(_ptr(q), _ptr(k), _ptr(v), P, bounds, n, _ptr(out), _ptr(out_lse), B, S, H,
+                                          D, scale, code, ctypes.c_void_p(_stream(q)))
+    _check(st, "cp_ring_sim_fused_ulysses")
+    return out, out_lse
+
+
+def ring_anything_gather(srcs, chunk_bounds: Sequence[int], max_len: Optional[int] = None, dsts=None):
+    """Ring Anything pad -> all-gather buffers of the ``[B, S, H, D]`` tensors ``srcs``:
+    each returned tensor is ``[n, B, max_len, H, D]`` with block c in ``[c, :, :len_c]``
+    and zeros after it (``max_len`` defaults to the longest block)."""
+    srcs = list(srcs)
+    if not srcs:
+        raise ValueError("need at least one tensor")
+    ref = srcs[0]
+    for t in srcs:
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or not t.is_contiguous() or t.dim() != 4 \
+                or t.shape != ref.shape or t.dtype != ref.dtype or t.device != ref.device:
+            raise ValueError("sources must be contiguous 4-D CUDA tensors of one shape, dtype and device")
+    if ref.element_size() not in (2, 4):
+        raise ValueError("elements must be 2 or 4 bytes")
+    B, S, H, D = ref.shape
+    n = len(chunk_bounds) - 1
+    if n < 1:
+        raise ValueError("chunk_bounds needs at least two entries")
+    lens = [int(b) - int(a) for a, b in zip(chunk_bounds[:-1], chunk_bounds[1:])]
+    if max_len is None:
+        max_len = max(lens)
+    if dsts is None:
+        dsts = [torch.empty((n, B, max_len, H, D), dtype=ref.dtype, device=ref.device) for _ in srcs]
+    dsts = list(dsts)
+    cnt = len(srcs)
+    sp = (ctypes.c_void_p * cnt)(*[t.data_ptr() for t in srcs])
+    dp = (ctypes.c_void_p * cnt)(*[t.data_ptr() for t in dsts])
+    bounds = (ctypes.c_int * (n + 1))(*[int(c) for c in chunk_bounds])
+    st = load().cp_ring_anything_gather(sp, dp, cnt, bounds, n, int(max_len), B, S, H, D, ref.element_size(),
+                                        ctypes.c_void_p(_stream(ref)))
+    _check(st, "cp_ring_anything_gather")
+    return dsts
 
 
 STATIC_SCRATCH_BYTES = 32 << 20

@@ -74,7 +74,7 @@ constexpr int kMaxChunks = 64;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // 2^x on the FMA pipe for one pair in kEmuEvery of a tile without masked keys (0: off):
 // n = rint(x) by the 1.5*2^23 shift, f = x - n in [-1/2, 1/2], 2^f by a degree-3 minimax
-// polynomial (relative error 7.5e-5; context_attention_dit_b200/exp2_poly_fit.py prints the
+// polynomial (relative error 7.5e-5; tests/exp2_poly_fit.py prints the
 // coefficients), 2^n added to the exponent.
 constexpr int kEmuEvery = 4;
 constexpr float kExp2C0 = 0.9999280571937561f;
@@ -89,10 +89,16 @@ struct AttnParams {
   int n_units;               // B * H * n_qt
   int tiles_per_unit;        // sum over blocks of ceil(len / kBN)
   float scale_log2;          // scale * log2(e)
-  void* out;                 // block c at out + c*out_chunk_stride elements, [B][Sq][H][D]
+  void* out;                 // block c at out + c*out_chunk_stride elements, row (b, s, h) at
+                             // b*o_sb + s*o_ss + h*D (dense BSHD: o_sb = Sq*H*D, o_ss = H*D)
   int out_f32;               // 1: fp32 output, 0: bf16 output
-  int out_v8;                // 1: out is 32-byte aligned (32-byte stores)
+  int out_v8;                // 1: every output row is 32-byte aligned (32-byte stores)
   long long out_chunk_stride;
+  long long o_sb, o_ss;      // element strides of the output's batch and sequence dimensions
+  int uly_p, uly_b;          // uly_p > 0: the attention ran on Ulysses head shards (batch
+                             // uly_p*uly_b, H = heads per shard) and each row goes to its place
+                             // in the sequence-sharded layout [uly_p][uly_b][Sq/uly_p][uly_p*H][D],
+                             // its LSE to [uly_b][uly_p*H][Sq] (the inverse exchange, fused)
   float* lse;                // block c at lse + c*lse_chunk_stride, [B][H][Sq]; may be null
   long long lse_chunk_stride;
   long long out_elems, lse_elems;  // extents of out and lse (checked in debug builds)
@@ -143,6 +149,31 @@ __device__ __forceinline__ UnitCoord decode_unit(int u, const AttnParams& p) {
   r.h = bh % p.H;
   r.b = bh / p.H;
   return r;
+}
+
+// Element offset of output row (b, s_row, h) of output block c, and the index of its LSE.
+template <int D>
+__device__ __forceinline__ long long out_row_offset(const AttnParams& p, int c, int b, int s_row, int h) {
+  const long long base = static_cast<long long>(c) * p.out_chunk_stride;
+  if (p.uly_p > 0) {
+    const int shard = b / p.uly_b, b0 = b - shard * p.uly_b;  // head shard, true batch
+    const int sp = p.Sq / p.uly_p;
+    const int ps = s_row / sp, s0 = s_row - ps * sp;           // sequence shard, its row
+    const long long hf = static_cast<long long>(p.uly_p) * p.H;
+    return base + ((static_cast<long long>(ps) * p.uly_b + b0) * sp + s0) * hf * D +
+           (static_cast<long long>(shard) * p.H + h) * D;
+  }
+  return base + b * p.o_sb + s_row * p.o_ss + static_cast<long long>(h) * D;
+}
+
+__device__ __forceinline__ long long lse_index(const AttnParams& p, int c, int b, int s_row, int h) {
+  const long long base = static_cast<long long>(c) * p.lse_chunk_stride;
+  if (p.uly_p > 0) {
+    const int shard = b / p.uly_b, b0 = b - shard * p.uly_b;
+    return base + (static_cast<long long>(b0) * p.uly_p * p.H + static_cast<long long>(shard) * p.H + h) * p.Sq +
+           s_row;
+  }
+  return base + (static_cast<long long>(b) * p.H + h) * p.Sq + s_row;
 }
 
 // Keys of a tile with `valid` keys that fall in half k (0..64).
@@ -574,8 +605,7 @@ __device__ __forceinline__ void store_row(const AttnParams& p, size_t o_off, con
 
 template <int D>
 __device__ __forceinline__ void write_empty_row(const AttnParams& p, int c, const UnitCoord& uc, int s_row) {
-  const size_t o_off = static_cast<size_t>(c) * p.out_chunk_stride +
-                       ((static_cast<size_t>(uc.b) * p.Sq + s_row) * p.H + uc.h) * D;
+  const size_t o_off = static_cast<size_t>(out_row_offset<D>(p, c, uc.b, s_row, uc.h));
   if (in_bounds(static_cast<long long>(o_off), D, p.out_elems)) {
     if (p.out_f32) {
       float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out) + o_off);
@@ -586,12 +616,10 @@ __device__ __forceinline__ void write_empty_row(const AttnParams& p, int c, cons
     }
   }
 #ifdef CP_DEBUG
-  const size_t li = static_cast<size_t>(c) * p.lse_chunk_stride + (static_cast<size_t>(uc.b) * p.H + uc.h) * p.Sq + s_row;
-  if (p.lse && in_bounds(static_cast<long long>(li), 1, p.lse_elems)) p.lse[li] = -INFINITY;
+  const long long li = lse_index(p, c, uc.b, s_row, uc.h);
+  if (p.lse && in_bounds(li, 1, p.lse_elems)) p.lse[li] = -INFINITY;
 #else
-  if (p.lse)
-    p.lse[static_cast<size_t>(c) * p.lse_chunk_stride + (static_cast<size_t>(uc.b) * p.H + uc.h) * p.Sq + s_row] =
-        -INFINITY;
+  if (p.lse) p.lse[lse_index(p, c, uc.b, s_row, uc.h)] = -INFINITY;
 #endif
 }
 
@@ -704,8 +732,7 @@ __device__ __forceinline__ void attn_epilogue(const AttnParams& p, uint8_t* smem
       const float lsum = s0.y * w0 + s1.y * w1;
       const float inv = 1.f / lsum;
       const float c0f = w0 * inv, c1f = w1 * inv;
-      const size_t o_off = static_cast<size_t>(c) * p.out_chunk_stride +
-                           ((static_cast<size_t>(uc.b) * p.Sq + s_row) * p.H + uc.h) * D;
+      const size_t o_off = static_cast<size_t>(out_row_offset<D>(p, c, uc.b, s_row, uc.h));
       // Read the whole merged O row into registers and release O before storing it: every
       // CTA reaches its block ends at about the same time, so a segment's stores run into
       // HBM bandwidth, and the next segment's first P.V must not wait for them.
@@ -737,14 +764,10 @@ __device__ __forceinline__ void attn_epilogue(const AttnParams& p, uint8_t* smem
         for (int cc = 0; cc < D / 32; ++cc) store_row<D>(p, o_off, *reinterpret_cast<const uint32_t(*)[32]>(r + cc * 32), cc);
       }
 #ifdef CP_DEBUG
-      const size_t li =
-          static_cast<size_t>(c) * p.lse_chunk_stride + (static_cast<size_t>(uc.b) * p.H + uc.h) * p.Sq + s_row;
-      if (row_ok && p.lse && in_bounds(static_cast<long long>(li), 1, p.lse_elems))
-        p.lse[li] = (mx + log2f(lsum)) * 0.69314718055994530942f;
+      const long long li = lse_index(p, c, uc.b, s_row, uc.h);
+      if (row_ok && p.lse && in_bounds(li, 1, p.lse_elems)) p.lse[li] = (mx + log2f(lsum)) * 0.69314718055994530942f;
 #else
-      if (row_ok && p.lse)
-        p.lse[static_cast<size_t>(c) * p.lse_chunk_stride + (static_cast<size_t>(uc.b) * p.H + uc.h) * p.Sq +
-              s_row] = (mx + log2f(lsum)) * 0.69314718055994530942f;
+      if (row_ok && p.lse) p.lse[lse_index(p, c, uc.b, s_row, uc.h)] = (mx + log2f(lsum)) * 0.69314718055994530942f;
 #endif
       ++nch;
     }

@@ -9,6 +9,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 
@@ -18,11 +19,12 @@
 #include "attn_fwd_sm100.cuh"
 #include "lse_merge.cuh"
 #include "peer.cuh"
+#include "ring_gather.cuh"
 #include "ulysses_permute.cuh"
 
 using namespace cpattn;
 
-static_assert(kMaxChunks == CP_MAX_CHUNKS, "chunk limit mismatch");
+static_assert(kMaxChunks == CP_MAX_CHUNKS && kGatherMaxChunks == CP_MAX_CHUNKS, "chunk limit mismatch");
 static_assert(kDevTimeout == CP_ERR_TIMEOUT && kDevBounds == CP_ERR_BOUNDS, "device status codes mismatch");
 static_assert(kPeerMax == CP_PEER_MAX && kPeerMergeMax == CP_PEER_MAX, "peer limit mismatch");
 static_assert(sizeof(cudaIpcMemHandle_t) == CP_IPC_HANDLE_BYTES, "IPC handle size mismatch");
@@ -80,19 +82,73 @@ cp_status device_info(DeviceInfo** out) {
   return CP_OK;
 }
 
-// 4-D map over a BSHD bf16 tensor: dims (D, H, S, B), box (64, 1, 128, 1), 128B swizzle.
-// Rows past S read as zeros.
-cp_status make_bshd_map(CUtensorMap* m, const void* base, int B, int S, int H, int D) {
+// Element strides of a [B][S][H][D] tensor's batch and sequence dimensions (the head stride
+// is D, the d stride 1).
+struct BsStrides {
+  long long sb, ss;
+};
+
+inline BsStrides dense(int S, int H, int D) {
+  return {static_cast<long long>(S) * H * D, static_cast<long long>(H) * D};
+}
+
+// Encoded tensor maps, keyed on everything that goes into the encoding.  Encoding three
+// maps costs microseconds of host time per call, which paces short launches; a map only
+// describes an address range and a shape, so reusing one for the same key is exact.
+struct MapKey {
+  int dev;
+  const void* base;
+  int B, S, H, D;
+  long long sb, ss;
+  bool operator==(const MapKey& o) const {
+    return dev == o.dev && base == o.base && B == o.B && S == o.S && H == o.H && D == o.D && sb == o.sb &&
+           ss == o.ss;
+  }
+};
+constexpr int kMapCacheSize = 64;
+struct MapCacheEntry {
+  MapKey key;
+  CUtensorMap map;
+  unsigned long long used = 0;  // 0: empty
+};
+std::mutex g_map_mutex;
+MapCacheEntry g_map_cache[kMapCacheSize];
+unsigned long long g_map_clock = 0;
+
+// 4-D map over a bf16 [B][S][H][D] tensor with element strides `st` (batch, sequence):
+// dims (D, H, S, B), box (64, 1, 128, 1), 128B swizzle.  Rows past S read as zeros.
+cp_status make_bshd_map(CUtensorMap* m, const void* base, int B, int S, int H, int D, BsStrides st) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return CP_ERR_CUDA;
+  if (B == 1) st.sb = st.ss * S;  // never used to address: any valid stride
+  const MapKey key{dev, base, B, S, H, D, st.sb, st.ss};
+  {
+    std::lock_guard<std::mutex> lock(g_map_mutex);
+    for (MapCacheEntry& e : g_map_cache)
+      if (e.used && e.key == key) {
+        e.used = ++g_map_clock;
+        *m = e.map;
+        return CP_OK;
+      }
+  }
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(S),
                         static_cast<cuuint64_t>(B)};
-  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2,
-                           static_cast<cuuint64_t>(S) * H * D * 2};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(st.ss) * 2,
+                           static_cast<cuuint64_t>(st.sb) * 2};
   cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(kBM), 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? CP_OK : CP_ERR_CUDA;
+  if (r != CUDA_SUCCESS) return CP_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_map_mutex);
+  MapCacheEntry* victim = &g_map_cache[0];
+  for (MapCacheEntry& e : g_map_cache)
+    if (e.used < victim->used) victim = &e;  // an empty entry (0) first, else the least recently used
+  victim->key = key;
+  victim->map = *m;
+  victim->used = ++g_map_clock;
+  return CP_OK;
 }
 
 cp_status check_attn_args(const void* q, const void* k, const void* v, const void* out, const float* lse, int B,
@@ -115,13 +171,29 @@ cp_status check_attn_args(const void* q, const void* k, const void* v, const voi
   return CP_OK;
 }
 
+// Layout of the attention's operands when they are not dense BSHD tensors.
+struct AttnLayout {
+  BsStrides q, kv, o;   // element strides (batch, sequence) of Q, of K and V, of the output
+  int uly_p = 0;        // > 0: output in the Ulysses sequence-sharded layout (see AttnParams)
+  int uly_b = 0;
+};
+
 // Launch the attention kernel over n_chunks K/V blocks given by `bounds` (host array).
+// `lay` == nullptr: Q, K, V and the output are dense BSHD tensors.
 cp_status launch_attn(const void* q, const void* k, const void* v, const int* bounds, int n_chunks, void* out,
                       int out_f32, long long out_chunk_stride, float* lse, long long lse_chunk_stride, int B, int H,
-                      int Sq, int Skv, int D, float scale, cudaStream_t stream, int fuse = 0) {
+                      int Sq, int Skv, int D, float scale, cudaStream_t stream, int fuse = 0,
+                      const AttnLayout* lay = nullptr) {
   DeviceInfo* dev = nullptr;
   cp_status st = device_info(&dev);
   if (st != CP_OK) return st;
+  AttnLayout dl;
+  if (!lay) {
+    dl.q = dense(Sq, H, D);
+    dl.kv = dense(Skv, H, D);
+    dl.o = dense(Sq, H, D);
+    lay = &dl;
+  }
   AttnParams p;
   std::memset(&p, 0, sizeof(p));
   p.B = B;
@@ -135,12 +207,23 @@ cp_status launch_attn(const void* q, const void* k, const void* v, const int* bo
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.out = out;
   p.out_f32 = out_f32;
-  p.out_v8 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0 ? 1 : 0;
   p.out_chunk_stride = out_chunk_stride;
+  p.o_sb = lay->o.sb;
+  p.o_ss = lay->o.ss;
+  p.uly_p = lay->uly_p;
+  p.uly_b = lay->uly_b;
+  {  // 32-byte stores need every row start 32-byte aligned
+    const long long eb = out_f32 ? 4 : 2;
+    const bool a32 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0 && (out_chunk_stride * eb) % 32 == 0 &&
+                     (lay->uly_p > 0 || ((lay->o.sb * eb) % 32 == 0 && (lay->o.ss * eb) % 32 == 0));
+    p.out_v8 = a32 ? 1 : 0;
+  }
   p.lse = lse;
   p.lse_chunk_stride = lse_chunk_stride;
-  {  // output extents: one [B][Sq][H][D] output (and [B][H][Sq] LSE) per written block
-    const long long one_o = static_cast<long long>(B) * Sq * H * D, one_l = static_cast<long long>(B) * H * Sq;
+  {  // output extents: one output (and [B][H][Sq] LSE) per written block
+    const long long one_o = lay->uly_p > 0 ? static_cast<long long>(B) * Sq * H * D
+                                           : (B - 1) * lay->o.sb + (Sq - 1) * lay->o.ss + static_cast<long long>(H) * D;
+    const long long one_l = static_cast<long long>(B) * H * Sq;
     const int n_out = (fuse || out_chunk_stride == 0) ? 1 : n_chunks;
     p.out_elems = out_chunk_stride ? out_chunk_stride * (n_out - 1) + one_o : one_o;
     p.lse_elems = lse_chunk_stride ? lse_chunk_stride * (n_out - 1) + one_l : one_l;
@@ -165,8 +248,10 @@ cp_status launch_attn(const void* q, const void* k, const void* v, const int* bo
   const int kv_rows = Skv > 0 ? Skv : 1;
   const void* kp = Skv > 0 ? k : q;
   const void* vp = Skv > 0 ? v : q;
-  if (make_bshd_map(&tq, q, B, Sq, H, D) != CP_OK || make_bshd_map(&tk, kp, B, Skv > 0 ? kv_rows : Sq, H, D) != CP_OK ||
-      make_bshd_map(&tv, vp, B, Skv > 0 ? kv_rows : Sq, H, D) != CP_OK)
+  const BsStrides kvs = Skv > 0 ? lay->kv : lay->q;
+  if (make_bshd_map(&tq, q, B, Sq, H, D, lay->q) != CP_OK ||
+      make_bshd_map(&tk, kp, B, Skv > 0 ? kv_rows : Sq, H, D, kvs) != CP_OK ||
+      make_bshd_map(&tv, vp, B, Skv > 0 ? kv_rows : Sq, H, D, kvs) != CP_OK)
     return CP_ERR_CUDA;
 
   const int grid = p.n_units < dev->num_sms ? p.n_units : dev->num_sms;
@@ -272,6 +357,45 @@ cp_status cp_attn_fwd(const void* q, const void* k, const void* v, void* out, fl
                      static_cast<cudaStream_t>(stream));
 }
 
+cp_status cp_attn_fwd_strided(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H,
+                              int Sq, int Skv, int D, long long q_sb, long long q_ss, long long kv_sb, long long kv_ss,
+                              long long o_sb, long long o_ss, float scale, cp_dtype out_dtype, void* stream) {
+  NvtxRange nvtx_range("cp_attn_fwd_strided");
+  cp_status st = check_attn_args(q, k, v, out, lse, B, H, Sq, Skv, D, scale, out_dtype);
+  if (st != CP_OK || B == 0 || H == 0 || Sq == 0) return st;
+  const long long row = static_cast<long long>(H) * D;
+  const long long eb = out_dtype == CP_F32 ? 4 : 2;
+  // Strides are positive; the batch stride matters only with more than one batch.
+  auto stride_bad = [&](long long sb, long long ss) { return ss <= 0 || (B > 1 && sb <= 0); };
+  if (stride_bad(q_sb, q_ss) || stride_bad(o_sb, o_ss) || (Skv > 0 && stride_bad(kv_sb, kv_ss)))
+    return CP_ERR_INVALID_ARG;
+  // TMA: bf16 input strides are multiples of 16 bytes (8 elements) and below 2^40 bytes.
+  auto tma_bad = [&](long long sb, long long ss) { return ss % 8 != 0 || (B > 1 && sb % 8 != 0); };
+  if (tma_bad(q_sb, q_ss) || (Skv > 0 && tma_bad(kv_sb, kv_ss))) return CP_ERR_MISALIGNED;
+  if (q_ss >= (1LL << 39) || q_sb >= (1LL << 39) || kv_ss >= (1LL << 39) || kv_sb >= (1LL << 39))
+    return CP_ERR_UNSUPPORTED;
+  // Output rows start on 16-byte boundaries and do not overlap (one dimension nests in the other).
+  if ((o_ss * eb) % 16 != 0 || (B > 1 && (o_sb * eb) % 16 != 0)) return CP_ERR_MISALIGNED;
+  {
+    long long s1 = o_ss, n1 = Sq, s2 = o_sb, n2 = B;
+    if (B > 1 && s2 < s1) {
+      std::swap(s1, s2);
+      std::swap(n1, n2);
+    }
+    const bool inner_ok = n1 == 1 || s1 >= row;
+    const bool outer_ok = n2 == 1 || s2 >= s1 * n1;
+    if (!(B == 1 ? (Sq == 1 || o_ss >= row) : (inner_ok && outer_ok && (n1 > 1 || s2 >= row))))
+      return CP_ERR_INVALID_ARG;
+  }
+  AttnLayout lay;
+  lay.q = {q_sb, q_ss};
+  lay.kv = {kv_sb, kv_ss};
+  lay.o = {o_sb, o_ss};
+  const int bounds[2] = {0, Skv};
+  return launch_attn(q, k, v, bounds, 1, out, out_dtype == CP_F32 ? 1 : 0, 0, lse, 0, B, H, Sq, Skv, D, scale,
+                     static_cast<cudaStream_t>(stream), 0, &lay);
+}
+
 cp_status cp_attn_merge(const float* partials, const float* lses, int n_chunks, void* out, float* out_lse, int B,
                         int H, int Sq, int D, cp_dtype out_dtype, void* stream) {
   NvtxRange nvtx_range("cp_attn_merge");
@@ -370,11 +494,11 @@ cp_status cp_ring_sim_static(const void* q, const void* k, const void* v, const 
   if (st != CP_OK || B == 0 || H == 0 || Sq == 0) return st;
   const size_t need = cp_ring_sim_workspace_size(n_chunks, B, H, Sq, D);
   if (need > CP_STATIC_SCRATCH_BYTES) return CP_ERR_UNSUPPORTED;
+  // The address look-up runs on every call, also one that needs no scratch (a single
+  // block), so that whichever call comes first on a device does the set-up.
   void* scratch = nullptr;
-  if (need > 0) {
-    st = static_scratch(&scratch);
-    if (st != CP_OK) return st;
-  }
+  st = static_scratch(&scratch);
+  if (st != CP_OK) return st;
   return cp_ring_sim(q, k, v, chunk_bounds, n_chunks, out, out_lse, B, H, Sq, Skv, D, scale, out_dtype, scratch,
                      need, stream);
 }
@@ -445,6 +569,96 @@ cp_status cp_ring_sim_fused(const void* q, const void* k, const void* v, const i
   if (st != CP_OK || B == 0 || H == 0 || Sq == 0) return st;
   return launch_attn(q, k, v, chunk_bounds, n_chunks, out, out_dtype == CP_F32 ? 1 : 0, 0, out_lse, 0, B, H, Sq, Skv,
                      D, scale, static_cast<cudaStream_t>(stream), 1);
+}
+
+cp_status cp_ring_sim_fused_ulysses(const void* q, const void* k, const void* v, int degree, const int* chunk_bounds,
+                                    int n_chunks, void* out, float* out_lse, int B, int S, int H, int D, float scale,
+                                    cp_dtype out_dtype, void* stream) {
+  NvtxRange nvtx_range("cp_ring_sim_fused_ulysses");
+  if (degree < 1 || B < 0 || S < 0 || H < 0) return CP_ERR_INVALID_ARG;
+  if (S % degree != 0 || H % degree != 0) return CP_ERR_NOT_DIVISIBLE;
+  cp_status st = check_bounds(chunk_bounds, n_chunks, S);
+  if (st != CP_OK) return st;
+  if (static_cast<long long>(degree) * B >= (1LL << 31)) return CP_ERR_UNSUPPORTED;
+  const int Bp = degree * B, Hp = H / degree;
+  st = check_attn_args(q, k, v, out, out_lse, Bp, Hp, S, S, D, scale, out_dtype);
+  if (st != CP_OK || B == 0 || H == 0 || S == 0) return st;
+  AttnLayout lay;
+  lay.q = lay.kv = lay.o = dense(S, Hp, D);
+  lay.uly_p = degree;
+  lay.uly_b = B;
+  return launch_attn(q, k, v, chunk_bounds, n_chunks, out, out_dtype == CP_F32 ? 1 : 0, 0, out_lse, 0, Bp, Hp, S, S,
+                     D, scale, static_cast<cudaStream_t>(stream), 1, &lay);
+}
+
+cp_status cp_ring_anything_gather(const void* const* srcs, void* const* dsts, int n_tensors, const int* chunk_bounds,
+                                  int n_chunks, int max_len, int B, int S, int H, int D, int elem_bytes,
+                                  void* stream) {
+  NvtxRange nvtx_range("cp_ring_anything_gather");
+  cp_status st = check_bounds(chunk_bounds, n_chunks, S);
+  if (st != CP_OK) return st;
+  if (B < 0 || H < 0 || D < 0 || max_len < 0) return CP_ERR_INVALID_ARG;
+  if (elem_bytes != 2 && elem_bytes != 4) return CP_ERR_UNSUPPORTED;
+  if (n_tensors < 1 || !srcs || !dsts) return CP_ERR_INVALID_ARG;
+  if (n_tensors > kGatherMaxTensors) return CP_ERR_UNSUPPORTED;
+  GatherArgs a;
+  std::memset(&a, 0, sizeof(a));
+  int longest = 0;
+  for (int c = 0; c < n_chunks; ++c) {
+    a.bounds[c] = chunk_bounds[c];
+    longest = std::max(longest, chunk_bounds[c + 1] - chunk_bounds[c]);
+  }
+  a.bounds[n_chunks] = chunk_bounds[n_chunks];
+  if (max_len < longest) return CP_ERR_INVALID_ARG;
+  if (B == 0 || H == 0 || D == 0 || max_len == 0) return CP_OK;
+  const long long row_bytes = static_cast<long long>(H) * D * elem_bytes;
+  const long long src_bytes = static_cast<long long>(B) * S * row_bytes;
+  const long long dst_bytes = static_cast<long long>(n_chunks) * B * max_len * row_bytes;
+  for (int t = 0; t < n_tensors; ++t) {
+    if (!dsts[t] || (S > 0 && !srcs[t])) return CP_ERR_INVALID_ARG;
+    if (!aligned16(dsts[t]) || (srcs[t] && !aligned16(srcs[t]))) return CP_ERR_MISALIGNED;
+    a.src[t] = srcs[t];
+    a.dst[t] = dsts[t];
+  }
+  // No destination may overlap a source or another destination.
+  for (int t = 0; t < n_tensors; ++t) {
+    const char* d0 = static_cast<const char*>(dsts[t]);
+    for (int u = 0; u < n_tensors; ++u) {
+      const char* s0 = static_cast<const char*>(srcs[u]);
+      if (s0 && s0 < d0 + dst_bytes && d0 < s0 + src_bytes) return CP_ERR_INVALID_ARG;
+      const char* e0 = static_cast<const char*>(dsts[u]);
+      if (u != t && e0 < d0 + dst_bytes && d0 < e0 + dst_bytes) return CP_ERR_INVALID_ARG;
+    }
+  }
+  const long long rows = static_cast<long long>(n_chunks) * B * max_len;  // destination rows per tensor
+  if (rows * n_tensors >= (1LL << 31) || row_bytes >= (1LL << 31)) return CP_ERR_UNSUPPORTED;
+  DeviceInfo* dev = nullptr;
+  st = device_info(&dev);
+  if (st != CP_OK) return st;
+  a.n_chunks = n_chunks;
+  a.B = B;
+  a.S = S;
+  a.max_len = max_len;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  auto launch = [&](auto tag) {
+    using V = decltype(tag);
+    const int row_vecs = static_cast<int>(row_bytes / sizeof(V));
+    const long long groups = (rows + kGatherRows - 1) / kGatherRows;
+    // About 8 resident blocks of rows per SM, each looping over its share of row groups.
+    const long long cap = static_cast<long long>(dev->num_sms) * 8;
+    const dim3 grid((row_vecs + kGatherThreads - 1) / kGatherThreads,
+                    static_cast<unsigned>(std::min<long long>(groups, std::max<long long>(1, cap))), n_tensors);
+    ring_anything_gather_kernel<V><<<grid, kGatherThreads, 0, cs>>>(a, row_vecs, rows);
+  };
+  if (row_bytes % 16 == 0)
+    launch(uint4{});
+  else if (row_bytes % 8 == 0)
+    launch(uint2{});
+  else if (row_bytes % 4 == 0)
+    launch(uint32_t{});
+  else
+    launch(uint16_t{});
+  return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
 }
 
 cp_status cp_ulysses_permute_n(const void* const* srcs, void* const* dsts, int n_tensors, int degree, int B, int S,

@@ -18,8 +18,12 @@
  *   - Layout "BSHD": [B][S][H][D] row-major, D fastest, densely packed.
  *   - LSE layout: float32 [B][H][Sq], natural logarithm.
  *   - Every pointer argument except chunk_bounds/bounds_out is a DEVICE pointer on
- *     the current CUDA device, owned by the caller; the library allocates no device
- *     memory and keeps no per-call state.  Device pointers must be 16-byte aligned,
+ *     the current CUDA device, owned by the caller.  No entry point allocates device
+ *     memory, with one exception: cp_peer_alloc, whose purpose is to allocate a buffer
+ *     that other processes can map.  Separately, loading the library creates one
+ *     file-scope device array of CP_STATIC_SCRATCH_BYTES (32 MiB) on every device that
+ *     runs its code (the scratch of cp_ring_sim_static), held until the process exits.
+ *     The library keeps no per-call state.  Device pointers must be 16-byte aligned,
  *     except LSE arrays (float32, read and written one element at a time: 4 bytes).
  *   - stream: a cudaStream_t passed as void*; NULL means the legacy default stream.
  *     All calls are asynchronous on that stream; inputs must stay alive until the
@@ -87,6 +91,31 @@ typedef enum { CP_BF16 = 0, CP_F32 = 1 } cp_dtype;
 CP_API cp_status cp_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
                       int B, int H, int Sq, int Skv, int D, float scale,
                       cp_dtype out_dtype, void* stream);
+
+/*
+ * cp_attn_fwd_strided - cp_attn_fwd on tensors that are views inside larger ones.
+ *
+ * Source: "Context parallelism", "Ring Attention": each ring step attends the local
+ * queries to one K/V block, which a caller often holds as a slice of a longer sequence
+ * (rows [c, c + Skv) of a [B][S][H][D] tensor), or Q/K/V as slices of a packed QKV
+ * tensor.  Same computation and output rules as cp_attn_fwd; only the addressing differs.
+ *
+ * Element (b, s, h, d) of q is at q + b*q_sb + s*q_ss + h*D + d (elements, not bytes);
+ * k and v share kv_sb/kv_ss; the output row (b, s, h) is at out + b*o_sb + s*o_ss + h*D.
+ * lse stays dense fp32 [B][H][Sq] (or NULL).
+ *   - Strides are > 0 (batch strides are ignored when B == 1).
+ *   - q/k/v strides are multiples of 8 elements (16 bytes, a TMA rule) and below 2^39;
+ *     output strides times the element size are multiples of 16 bytes.
+ *     Violations: CP_ERR_MISALIGNED (alignment) or CP_ERR_UNSUPPORTED (size).
+ *   - Output rows (H*D elements each) must not overlap: one of the two output
+ *     dimensions must nest inside the other (the smaller stride >= H*D, the larger >=
+ *     the smaller times its extent); otherwise CP_ERR_INVALID_ARG.  Inputs may overlap.
+ * Dense BSHD tensors (q_sb = Sq*H*D, q_ss = H*D, ...) give exactly cp_attn_fwd's result.
+ */
+CP_API cp_status cp_attn_fwd_strided(const void* q, const void* k, const void* v, void* out, float* lse,
+                                     int B, int H, int Sq, int Skv, int D, long long q_sb, long long q_ss,
+                                     long long kv_sb, long long kv_ss, long long o_sb, long long o_ss,
+                                     float scale, cp_dtype out_dtype, void* stream);
 
 /*
  * cp_attn_fwd_blocks - attention of q over every K/V block, without the merge.
@@ -162,6 +191,53 @@ CP_API cp_status cp_ring_sim_fused(const void* q, const void* k, const void* v, 
                             int n_chunks, void* out, float* out_lse, int B, int H, int Sq, int Skv,
                             int D, float scale, cp_dtype out_dtype, void* stream);
 
+/*
+ * cp_ring_sim_fused_ulysses - Ulysses x ring attention after the first exchange: the fused
+ * ring over K/V blocks on the head shards, writing the output in the sequence-sharded
+ * layout (the second all-to-all folded into the kernel's epilogue).
+ *
+ * Source: "Context parallelism", "Unified Attention": an all-to-all regroups heads and
+ * tokens, Ring Attention runs on the result, and the reverse all-to-all restores the
+ * token layout.  Here the ring is cp_ring_sim_fused (the running max/sum/output carried
+ * across blocks in TMEM, no partials) and each finished row is stored straight to its
+ * place in the token-sharded output, so the head-sharded output is never written.
+ * q, k, v:  bf16 head-sharded [degree][B][S][H/degree][D] (head shard p = heads
+ *           [p*H/degree, (p+1)*H/degree)), as produced by cp_ulysses_permute direction 0.
+ * chunk_bounds: HOST int[n_chunks+1] over [0, S], as cp_ring_sim with Skv = S.
+ * out:      [degree][B][S/degree][H][D], bf16 or fp32 (out_dtype): the layout of
+ *           cp_ulysses_permute direction 1 applied to the attention output.
+ * out_lse:  fp32 [B][H][S] natural log, or NULL.
+ * Errors: S or H not divisible by degree -> CP_ERR_NOT_DIVISIBLE; otherwise as
+ * cp_ring_sim_fused.  Allocates nothing.  The result equals cp_usp_sim's up to fp32
+ * rounding order (the merge runs inside the kernel).
+ */
+CP_API cp_status cp_ring_sim_fused_ulysses(const void* q, const void* k, const void* v, int degree,
+                                           const int* chunk_bounds, int n_chunks, void* out, float* out_lse,
+                                           int B, int S, int H, int D, float scale, cp_dtype out_dtype,
+                                           void* stream);
+
+/*
+ * cp_ring_anything_gather - the Ring Anything pad -> all-gather buffer, built on one GPU.
+ *
+ * Source: "Context parallelism", "Ring Anything Attention": ranks whose K/V blocks have
+ * different lengths pad their block to the longest, all-gather the padded blocks, and
+ * slice each gathered block back to its true length before attention.  This call builds
+ * the gathered buffer of every tensor from the unsharded one:
+ *   dst[c][b][r][h][d] = src[b][chunk_bounds[c] + r][h][d]   for r < len_c,
+ *   dst[c][b][r][h][d] = 0                                    for len_c <= r < max_len,
+ * with len_c = chunk_bounds[c+1] - chunk_bounds[c].  Block c's true-length slice is the
+ * [B][len_c][H][D] view at dst + c*B*max_len*H*D with batch stride max_len*H*D and sequence
+ * stride H*D, which cp_attn_fwd_strided attends in place.  The copy is exact (bit for bit).
+ * srcs:  n_tensors (1..8) device pointers, each [B][S][H][D] with elem_bytes-byte elements.
+ * dsts:  n_tensors device pointers, each [n_chunks][B][max_len][H][D] (written); no
+ *        destination may overlap a source or another destination (CP_ERR_INVALID_ARG).
+ * chunk_bounds: HOST int[n_chunks+1] over [0, S] as cp_ring_sim; max_len >= the longest
+ *        block (CP_ERR_INVALID_ARG otherwise).  elem_bytes 2 or 4.  Pointers 16-byte aligned.
+ */
+CP_API cp_status cp_ring_anything_gather(const void* const* srcs, void* const* dsts, int n_tensors,
+                                         const int* chunk_bounds, int n_chunks, int max_len, int B, int S,
+                                         int H, int D, int elem_bytes, void* stream);
+
 /* Size in bytes of the workspace cp_usp_sim needs (0 for invalid sizes or H % degree != 0). */
 CP_API size_t cp_usp_sim_workspace_size(int degree, int n_chunks, int B, int S, int H, int D,
                                         cp_dtype out_dtype);
@@ -195,20 +271,22 @@ CP_API cp_status cp_usp_sim(const void* q, const void* k, const void* v, int deg
 /*
  * cp_ring_sim_static - cp_ring_sim for callers that cannot allocate device memory.
  *
- * The pages have no counterpart to this call; it exists for users of this library
- * whose code may not call cudaMalloc (or any allocator) when they attend: code
- * running inside another framework's memory pool, during CUDA stream capture,
- * or in a real-time loop that must not allocate.  It computes exactly what
- * cp_ring_sim computes, with the same arguments minus workspace/ws_bytes: the
- * per-block fp32 partials and LSEs live in one file-scope device array of
- * CP_STATIC_SCRATCH_BYTES (32 MiB) that every GPU which loads the library keeps
- * until the process exits.  The call allocates nothing.
+ * The pages have no counterpart to this call.  It exists for callers of this library
+ * that may not allocate device memory at the point where they attend: code that runs
+ * inside another framework's memory pool or under a fixed memory budget, where a
+ * cudaMalloc would bypass the pool's accounting or fail, and real-time loops where an
+ * allocation's latency (and the synchronisation cudaMalloc/cudaFree can imply) is not
+ * allowed.  It computes exactly what cp_ring_sim computes, with the same arguments
+ * minus workspace/ws_bytes: the per-block fp32 partials and LSEs live in one
+ * file-scope device array of CP_STATIC_SCRATCH_BYTES (32 MiB) that every GPU which
+ * loads the library keeps until the process exits.  The call allocates nothing.
  *
  * - Sizes: if cp_ring_sim_workspace_size(n_chunks, B, H, Sq, D) exceeds
  *   CP_STATIC_SCRATCH_BYTES the call returns CP_ERR_UNSUPPORTED and launches nothing.
- * - Set-up: the first call on a device looks up the array's device address with
- *   that device current (cudaGetSymbolAddress); make that first call before any
- *   stream capture.  A failed look-up returns CP_ERR_CUDA.
+ * - Set-up: the first call on a device with non-empty sizes (B, H, Sq > 0) looks up
+ *   the array's device address with that device current (cudaGetSymbolAddress), also
+ *   when it needs no scratch (a single block); make that first call before any stream
+ *   capture.  A failed look-up returns CP_ERR_CUDA.
  * - Sharing: every call on every stream of a device uses the same array.  Calls
  *   that overlap on the GPU (different streams, no ordering) race and corrupt each
  *   other's results; order them on one stream or with events.  The array keeps the

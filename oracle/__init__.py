@@ -17,8 +17,9 @@ message-passing all-to-all.  No function here is "parity unpinned".
 """
 
 from .attention import attention, merge, ring, attention_rows
+from .ring_anything import ring_anything_gather, ring_anything_slice
 from .ulysses import ulysses_anything_fwd, ulysses_anything_inv, ulysses_fwd, ulysses_inv
 from .usp import usp
 
-__all__ = ["attention", "merge", "ring", "attention_rows", "ulysses_fwd", "ulysses_inv", "ulysses_anything_fwd",
+__all__ = ["attention", "merge", "ring", "attention_rows", "ring_anything_gather", "ring_anything_slice", "ulysses_fwd", "ulysses_inv", "ulysses_anything_fwd",
            "ulysses_anything_inv", "usp"]

@@ -37,6 +37,11 @@ def run():
         o, lse, _ = binding.ring_sim(q, k, v, bounds)
         record(f"ring_{bounds}", o, lse)
         record(f"ring_fused_{bounds}", *binding.ring_sim_fused(q, k, v, bounds, out_dtype=torch.float32))
+    # The allocation-free ring on a shape whose partials and LSEs nearly fill the static
+    # array (2 blocks x 4 heads x 8128 rows: 33,552,384 of 33,554,432 bytes).
+    qs, ks, vs = (t.cuda() for t in make_qkv(1, 4, 8128, 300, 128, seed=10))
+    assert binding.ring_workspace_size(2, 1, 4, 8128, 128) > binding.STATIC_SCRATCH_BYTES - 4096
+    record("ring_static_near_limit", *binding.ring_sim_static(qs, ks, vs, [0, 150, 300]))
     P, B, S, H, D = 4, 2, 384, 8, 128
     x = [t.cuda() for t in make_qkv(P * B, H // P, S, S, D, seed=5)]
     parts, lses = binding.attn_fwd_blocks(*x, [0, 100, 101, 384])

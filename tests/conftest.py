@@ -28,3 +28,19 @@ def lib():
     from context_attention_dit_b200 import binding
 
     return binding.load()
+
+
+_PARITY_LINES = []
+
+
+@pytest.fixture
+def parity_report():
+    """Record a line for the session's parity summary (printed even under -q)."""
+    return _PARITY_LINES.append
+
+
+def pytest_terminal_summary(terminalreporter):
+    if _PARITY_LINES:
+        terminalreporter.section("parity summary")
+        for line in _PARITY_LINES:
+            terminalreporter.write_line(line)

@@ -7,7 +7,7 @@ error over [-1/2, 1/2].  The minimax problem is solved on a dense grid as a line
 program (minimise t subject to |p(f_i) - 2^f_i| <= t * 2^f_i), then the coefficients are
 rounded to float32 and the error of the float32 Horner evaluation is measured.
 
-Run ``python -m context_attention_dit_b200.exp2_poly_fit`` to print the
+Run ``python -m tests.exp2_poly_fit`` to print the
 coefficients written into ``attn_fwd_sm100.cuh`` (kExp2C0..kExp2C3).
 """
 

@@ -385,3 +385,81 @@ def pin_anything_reduces_to_even(ulysses_anything_fwd, ulysses_fwd):
     any_ = ulysses_anything_fwd([stacked[p] for p in range(P)], _near_even(S, P), _near_even(H, P))
     for q in range(P):
         assert np.array_equal(np.asarray(any_[q]), np.asarray(even[q]))
+
+
+# --------------------------------------------------------------------------- Ring Anything gather
+
+def load_golden_gather():
+    """tests/golden/ring_anything_gather_s5.txt: hand-written gathered buffer (block, row, value)."""
+    rows = []
+    with open(os.path.join(GOLDEN, "ring_anything_gather_s5.txt")) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if line:
+                rows.append(tuple(int(t) for t in line.split()))
+    return rows
+
+
+def pin_gather_golden(ring_anything_gather):
+    """B=1, S=5, H=D=1, blocks 2/1/2 padded to 2; token t holds 10*t + 1."""
+    x = np.array([10 * t + 1 for t in range(5)], dtype=np.int64).reshape(1, 5, 1, 1)
+    out = ring_anything_gather(x, [0, 2, 3, 5], 2)
+    rows = load_golden_gather()
+    assert np.asarray(out).shape == (3, 1, 2, 1, 1)
+    for c, r, val in rows:
+        assert int(out[c, 0, r, 0, 0]) == val, f"golden block {c} row {r}"
+    assert len(rows) == 3 * 2
+
+
+def _pad_then_allgather(x, bounds, max_len):
+    """The pages' procedure by ranks: rank c holds rows [c_c, c_{c+1}), pads them at the
+    end to max_len with zero rows, and the all-gather stacks every rank's padded block."""
+    blocks = [x[:, bounds[c]:bounds[c + 1]] for c in range(len(bounds) - 1)]
+    padded = [np.pad(blk, ((0, 0), (0, max_len - blk.shape[1]), (0, 0), (0, 0))) for blk in blocks]
+    return np.stack(padded)
+
+
+GATHER_CASES = [
+    # (B, S, H, D, bounds, max_len)
+    (1, 7, 2, 3, [0, 3, 5, 7], 3),                # uneven
+    (2, 9, 3, 2, [0, 0, 4, 9], 5),                # an empty block
+    (2, 8, 1, 4, [0, 2, 4, 6, 8], 2),             # even: no padding rows
+    (3, 17, 2, 1, [0, 5, 9, 13, 17], 7),          # FLUX-1008-like split, extra padding
+]
+
+
+def pin_gather_per_rank(ring_anything_gather):
+    """The index map equals padding on every rank followed by an all-gather (bit-exact)."""
+    r = _rng(31)
+    for B, S, H, D, bounds, max_len in GATHER_CASES:
+        x = r.standard_normal((B, S, H, D)).astype(np.float32)
+        assert np.array_equal(np.asarray(ring_anything_gather(x, bounds, max_len)),
+                              _pad_then_allgather(x, bounds, max_len)), (B, S, bounds)
+
+
+def pin_gather_slice_roundtrip(ring_anything_gather, ring_anything_slice):
+    """Cutting the gathered blocks back to their true lengths and joining them along the
+    sequence restores the input exactly; every padding row is zero."""
+    r = _rng(32)
+    for B, S, H, D, bounds, max_len in GATHER_CASES:
+        x = r.standard_normal((B, S, H, D)) + 3.0  # no zero rows in the data
+        g = np.asarray(ring_anything_gather(x, bounds, max_len))
+        blocks = ring_anything_slice(g, bounds)
+        assert np.array_equal(np.concatenate([np.asarray(b) for b in blocks], axis=1), x), (B, S, bounds)
+        for c in range(len(bounds) - 1):
+            assert not np.any(g[c, :, bounds[c + 1] - bounds[c]:]), f"padding of block {c} not zero"
+
+
+def pin_gather_ring_equals_unsplit(attention, merge, ring_anything_gather, ring_anything_slice):
+    """Attention over the sliced gathered blocks, merged by LSE, equals unsplit attention
+    (fp64, 1e-12): the padding has no numerical effect once sliced off."""
+    r = _rng(33)
+    B, S, H, D = 2, 11, 2, 4
+    q, k, v = (r.standard_normal((B, S, H, D)) for _ in range(3))
+    bounds, max_len = [0, 4, 7, 11], 6
+    kb = ring_anything_slice(ring_anything_gather(k, bounds, max_len), bounds)
+    vb = ring_anything_slice(ring_anything_gather(v, bounds, max_len), bounds)
+    parts = [attention(q, kc, vc, 0.7) for kc, vc in zip(kb, vb)]
+    o, lse = merge(np.stack([p[0] for p in parts]), np.stack([p[1] for p in parts]))
+    o_full, lse_full = attention(q, k, v, 0.7)
+    assert np.allclose(o, o_full, rtol=0, atol=1e-12) and np.allclose(lse, lse_full, rtol=0, atol=1e-12)

@@ -342,3 +342,58 @@ def test_peer_bindings_reject_bad_arguments_before_the_library():
         binding.attn_merge_push(torch.zeros(1, 1, 4, 1, 64), torch.zeros(1, 1, 1, 4), [1 << 20, 2 << 20], 0)
     with pytest.raises(ValueError):
         binding.ulysses_anything_permute_n([torch.zeros(8)], 2, [0, 1, 2], [0, 1, 2], 1, 2, 2, 2, 0)
+
+
+def test_attn_fwd_strided_checks_before_cuda(lib):
+    """Strides and the output's row layout are checked on the host, before any CUDA call."""
+    vp = ctypes.c_void_p
+    q, k, v, o = vp(1 << 20), vp(2 << 20), vp(3 << 20), vp(4 << 20)
+    B, H, S, D = 2, 3, 16, 64
+    row = H * D
+
+    def call(q_sb=S * row, q_ss=row, kv_sb=S * row, kv_ss=row, o_sb=S * row, o_ss=row, dt=0, b=B):
+        return lib.cp_attn_fwd_strided(q, k, v, o, None, b, H, S, S, D, q_sb, q_ss, kv_sb, kv_ss, o_sb, o_ss, 0.1,
+                                       dt, None)
+
+    assert call(q_ss=0) == I.CP_ERR_INVALID_ARG
+    assert call(kv_sb=-8) == I.CP_ERR_INVALID_ARG
+    assert call(o_ss=-row) == I.CP_ERR_INVALID_ARG
+    assert call(q_ss=row + 4) == I.CP_ERR_MISALIGNED                  # TMA: 16-byte strides
+    assert call(kv_sb=S * row + 4) == I.CP_ERR_MISALIGNED
+    assert call(o_ss=row + 4) == I.CP_ERR_MISALIGNED                  # bf16 rows on 16-byte bounds
+    assert call(o_ss=row + 4, dt=1) != I.CP_ERR_MISALIGNED            # fp32: 4 elements are 16 bytes
+    assert call(q_ss=1 << 39) == I.CP_ERR_UNSUPPORTED
+    assert call(o_ss=row - 8) == I.CP_ERR_INVALID_ARG                 # output rows overlap
+    assert call(o_sb=row * 4) == I.CP_ERR_INVALID_ARG                 # batches overlap along the sequence
+    # An interleaved output (the sequence outermost, batches side by side) passes the checks
+    # and reaches CUDA, which is absent here: CP_ERR_CUDA, not an argument error.
+    assert call(o_sb=row, o_ss=B * row) not in (I.CP_ERR_INVALID_ARG, I.CP_ERR_MISALIGNED, I.CP_ERR_UNSUPPORTED)
+    assert call(o_sb=0, b=1) not in (I.CP_ERR_INVALID_ARG, I.CP_ERR_MISALIGNED)  # batch stride unused for B = 1
+    assert lib.cp_attn_fwd_strided(None, None, None, None, None, 0, H, S, S, D, 0, 0, 0, 0, 0, 0, 0.1, 0,
+                                   None) == I.CP_OK                   # empty batch: nothing to do
+
+
+def test_ring_sim_fused_ulysses_checks_before_cuda(lib):
+    p = ctypes.c_void_p(1 << 20)
+    call = lambda deg, S, H, b: lib.cp_ring_sim_fused_ulysses(  # noqa: E731
+        p, p, p, deg, _bounds(*b), len(b) - 1, p, None, 1, S, H, 64, 0.1, 0, None)
+    assert call(3, 16, 6, (0, 16)) == I.CP_ERR_NOT_DIVISIBLE    # S % degree
+    assert call(4, 16, 6, (0, 16)) == I.CP_ERR_NOT_DIVISIBLE    # H % degree
+    assert call(2, 16, 4, (0, 9, 15)) == I.CP_ERR_INVALID_ARG   # bounds do not span [0, S]
+    assert call(0, 16, 4, (0, 16)) == I.CP_ERR_INVALID_ARG
+
+
+def test_ring_anything_gather_checks_before_cuda(lib):
+    vp = ctypes.c_void_p
+    srcs, dsts = (vp * 2)(1 << 20, 2 << 20), (vp * 2)(3 << 20, 4 << 20)
+    call = lambda s, d, n, b, max_len, eb=2: lib.cp_ring_anything_gather(  # noqa: E731
+        s, d, n, _bounds(*b), len(b) - 1, max_len, 1, b[-1], 2, 8, eb, None)
+    assert call(srcs, dsts, 2, (0, 3, 5), 2) == I.CP_ERR_INVALID_ARG      # max_len below the longest block
+    assert call(srcs, dsts, 2, (0, 3, 2, 5), 3) == I.CP_ERR_INVALID_ARG   # decreasing bounds
+    assert call(srcs, dsts, 2, (0, 3, 5), 3, eb=8) == I.CP_ERR_UNSUPPORTED
+    assert call(srcs, dsts, 9, (0, 3, 5), 3) == I.CP_ERR_UNSUPPORTED      # more than 8 tensors
+    assert call(srcs, dsts, 0, (0, 3, 5), 3) == I.CP_ERR_INVALID_ARG
+    assert call(srcs, (vp * 2)(3 << 20, 1 << 20), 2, (0, 3, 5), 3) == I.CP_ERR_INVALID_ARG  # dst on a source
+    assert call(srcs, (vp * 2)(3 << 20, 3 << 20), 2, (0, 3, 5), 3) == I.CP_ERR_INVALID_ARG  # dsts overlap
+    assert call(srcs, (vp * 2)(3 << 20, (4 << 20) + 8), 2, (0, 3, 5), 3) == I.CP_ERR_MISALIGNED
+    assert call(srcs, dsts, 2, (0, 0, 0), 0) == I.CP_OK                   # no rows: nothing to copy

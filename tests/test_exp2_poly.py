@@ -7,7 +7,7 @@ import re
 
 import numpy as np
 
-from context_attention_dit_b200 import exp2_poly_fit
+from tests import exp2_poly_fit
 
 KERNEL = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "context_attention_dit_b200",
                       "csrc", "attn_fwd_sm100.cuh")

@@ -83,6 +83,14 @@ USP_MUTANTS = [
 ]
 
 
+GATHER_MUTANTS = [
+    ("block start off by one", "out[c, b, r] = x[b, lo + r]", "out[c, b, r] = x[b, min(lo + r + 1, S - 1)]"),
+    ("padding in front of the block", "out[c, b, r] = x[b, lo + r]", "out[c, b, max_len - (hi - lo) + r] = x[b, lo + r]"),
+    ("blocks gathered in reverse rank order", "out[c, b, r] = x[b, lo + r]", "out[n - 1 - c, b, r] = x[b, lo + r]"),
+    ("slice keeps the padding", "gathered[c, :, :bounds[c + 1] - bounds[c]]", "gathered[c]"),
+]
+
+
 @pytest.mark.parametrize("name,old,new", ATTN_MUTANTS, ids=[m[0] for m in ATTN_MUTANTS])
 def test_attention_mutant_is_caught(name, old, new):
     ns = _load_mutant("attention.py", old, new)
@@ -123,4 +131,17 @@ def test_ulysses_anything_mutant_is_caught(name, old, new):
     ns = _load_mutant("ulysses.py", old, new)
     checks = [lambda: pins.pin_anything_origin(ns["ulysses_anything_fwd"], oracle.ulysses_anything_inv),
               lambda: pins.pin_anything_reduces_to_even(ns["ulysses_anything_fwd"], oracle.ulysses_fwd)]
+    assert any(_fails(c) for c in checks), f"mutant '{name}' passed every pin"
+
+
+@pytest.mark.parametrize("name,old,new", GATHER_MUTANTS, ids=[m[0] for m in GATHER_MUTANTS])
+def test_ring_anything_gather_mutant_is_caught(name, old, new):
+    import oracle
+
+    ns = _load_mutant("ring_anything.py", old, new)
+    checks = [lambda: pins.pin_gather_golden(ns["ring_anything_gather"]),
+              lambda: pins.pin_gather_per_rank(ns["ring_anything_gather"]),
+              lambda: pins.pin_gather_slice_roundtrip(ns["ring_anything_gather"], ns["ring_anything_slice"]),
+              lambda: pins.pin_gather_ring_equals_unsplit(oracle.attention, oracle.merge, ns["ring_anything_gather"],
+                                                          ns["ring_anything_slice"])]
     assert any(_fails(c) for c in checks), f"mutant '{name}' passed every pin"

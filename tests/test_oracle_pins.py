@@ -81,3 +81,20 @@ def test_bf16_inputs_widen_exactly():
     o2, l2 = oracle.attention(q.float().numpy(), k.float().numpy(), v.float().numpy(), 0.25)
     assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
     assert q.dtype == torch.bfloat16
+
+
+def test_ring_anything_gather_golden():
+    pins.pin_gather_golden(oracle.ring_anything_gather)
+
+
+def test_ring_anything_gather_per_rank():
+    pins.pin_gather_per_rank(oracle.ring_anything_gather)
+
+
+def test_ring_anything_gather_slice_roundtrip():
+    pins.pin_gather_slice_roundtrip(oracle.ring_anything_gather, oracle.ring_anything_slice)
+
+
+def test_ring_anything_gather_ring_equals_unsplit():
+    pins.pin_gather_ring_equals_unsplit(oracle.attention, oracle.merge, oracle.ring_anything_gather,
+                                        oracle.ring_anything_slice)
