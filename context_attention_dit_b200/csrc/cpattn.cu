@@ -10,6 +10,7 @@
 #include <cmath>
 #include <cstdint>
 #include <algorithm>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -17,6 +18,7 @@
 #include <nvtx3/nvToolsExt.h>
 
 #include "attn_fwd_sm100.cuh"
+#include "attn_pair_sm100.cuh"
 #include "lse_merge.cuh"
 #include "peer.cuh"
 #include "ring_gather.cuh"
@@ -38,7 +40,18 @@ struct DeviceInfo {
   int num_sms = 0;
   int* status = nullptr;  // device address of g_cp_status
   bool attn_attr_set[2] = {false, false};
+  bool pair_attr_set[2] = {false, false};
 };
+
+// Which attention kernel runs: the one-Q-tile kernel (attn_fwd_sm100) unless
+// CPATTN_ATTN_KERNEL=pair selects the two-Q-tile kernel (attn_pair_sm100).
+bool use_pair_kernel() {
+  static const bool pair = [] {
+    const char* e = std::getenv("CPATTN_ATTN_KERNEL");
+    return e && std::strcmp(e, "pair") == 0;
+  }();
+  return pair;
+}
 
 std::mutex g_mutex;
 DeviceInfo g_dev[kMaxDevices];
@@ -254,6 +267,30 @@ cp_status launch_attn(const void* q, const void* k, const void* v, const int* bo
       make_bshd_map(&tv, vp, B, Skv > 0 ? kv_rows : Sq, H, D, kvs) != CP_OK)
     return CP_ERR_CUDA;
 
+  if (use_pair_kernel()) {
+    const int units = B * H * ((p.n_qt + 1) / 2);
+    const int grid = units < dev->num_sms ? units : dev->num_sms;
+    if (D == 128) {
+      using L = pair::Smem<128>;
+      if (!dev->pair_attr_set[1]) {
+        if (cudaFuncSetAttribute(pair::attn_pair_sm100_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 L::kRequest) != cudaSuccess)
+          return CP_ERR_CUDA;
+        dev->pair_attr_set[1] = true;
+      }
+      pair::attn_pair_sm100_kernel<128><<<grid, pair::kThreads, L::kRequest, stream>>>(tq, tk, tv, p);
+    } else {
+      using L = pair::Smem<64>;
+      if (!dev->pair_attr_set[0]) {
+        if (cudaFuncSetAttribute(pair::attn_pair_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 L::kRequest) != cudaSuccess)
+          return CP_ERR_CUDA;
+        dev->pair_attr_set[0] = true;
+      }
+      pair::attn_pair_sm100_kernel<64><<<grid, pair::kThreads, L::kRequest, stream>>>(tq, tk, tv, p);
+    }
+    return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+  }
   const int grid = p.n_units < dev->num_sms ? p.n_units : dev->num_sms;
   if (D == 128) {
     using L = AttnSmem<128>;
