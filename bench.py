@@ -210,7 +210,7 @@ def run_ours(args):
     flush_mib = flush_buf.numel() * 4 >> 20
 
     def flush_l2():
-        torch.sum(flush_buf, dtype=torch.float32, out=flush_sink)
+        torch.sum(flush_buf, dim=0, out=flush_sink)
     scale = w.scale
     flop = w.flop
     launches_per_step = 1 + 1 + 1  # exchange of Q, K, V; attention; merge fused with the inverse exchange

@@ -48,7 +48,9 @@ constexpr int kEpilogueWarp0 = 12;
 constexpr int kSoftmaxRegs = 200;
 constexpr int kControlRegs = 48;
 constexpr int kEpilogueRegs = 64;
-static_assert(2 * kSoftmaxRegs + kControlRegs + kEpilogueRegs == 4 * 128, "register split must use the launch budget");
+constexpr int kLaunchRegs = 65536 / kThreads;  // registers per thread at launch (128)
+static_assert(2 * kSoftmaxRegs + kControlRegs + kEpilogueRegs == 4 * kLaunchRegs,
+              "register split must use the launch budget");
 constexpr int kTmemO = 256;           // O_i at kTmemO + 128 i
 
 template <int D>
@@ -574,10 +576,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp >= kEpilogueWarp0) {
-    regs_increase<kEpilogueRegs>();
+    regs_set<kEpilogueRegs, kLaunchRegs>();
     epilogue<D>(p, smem, bars, tmem, abort_flag);
   } else if (warp >= 8) {
-    regs_decrease<kControlRegs>();
+    regs_set<kControlRegs, kLaunchRegs>();
     if (warp == kProducerWarp) {
       if ((threadIdx.x & 31) == 0) producer_qk<D>(&tm_q, &tm_k, p, smem, bars, abort_flag);
     } else if (warp == kVProducerWarp) {
@@ -589,7 +591,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else {
-    regs_increase<kSoftmaxRegs>();
+    regs_set<kSoftmaxRegs, kLaunchRegs>();
     softmax<D>(p, smem, bars, tmem, abort_flag);
   }
 

@@ -344,6 +344,16 @@ template <int N>
 __device__ __forceinline__ void regs_decrease() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
+// Set the warpgroup's register budget to N from the launch budget `kLaunch`: .inc only
+// raises and .dec only lowers it (the other direction is an illegal instruction).
+template <int N, int kLaunch>
+__device__ __forceinline__ void regs_set() {
+  static_assert(N % 8 == 0 && N >= 24 && N <= 256, "setmaxnreg takes a multiple of 8 in [24, 256]");
+  if constexpr (N > kLaunch)
+    regs_increase<N>();
+  else if constexpr (N < kLaunch)
+    regs_decrease<N>();
+}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x (low half) = lo
