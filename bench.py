@@ -1,11 +1,15 @@
 """Benchmark of the context-parallel attention hot path on B200.
 
 One step = the whole hot path on the FLUX.1-dev 1024x1024 joint-attention shape
-(B=1, H=24, S=4608, D=128, bf16, QK-normed synthetic inputs):
+(B=1, H=24, S=4608, D=128, bf16, QK-normed synthetic inputs), in two launches:
   1. Ulysses degree-8 exchange of Q, K and V (sequence-sharded -> head-sharded),
-  2. ring attention over 8 K/V blocks of 576 keys on the head-sharded tensors
-     (blockwise tcgen05 attention writing fp32 partials + LSE, then the LSE merge),
-  3. inverse Ulysses exchange of O.
+  2. ring attention over 8 K/V blocks of 576 keys on the head-sharded tensors, each
+     block merged into the running output by LSE rescaling in TMEM (the ring's merge,
+     pairwise in ring order), each finished row stored to its sequence-sharded place
+     (the inverse Ulysses exchange of O).
+The same path in three launches (blockwise attention writing every block's fp32
+partial and LSE to HBM, then the LSE merge kernel fused with the inverse exchange) is
+timed beside it and reported under "kernels".
 Metric: attention TFLOP/s = 4*B*H*S*S*D per step / step time (device time, CUDA
 events, L2 flushed between steps).  Also reported: the dominant kernel's roofline,
 the single-block (ring-1) attention kernel, merge and permute GB/s, the fp64 CPU
@@ -34,7 +38,7 @@ WORKLOAD = "flux_1024_ring8_ulysses8"
 METRIC = "attention TFLOP/s (4*B*H*Sq*Skv*D) and % of B200 BF16 peak; merge/permute GB/s"
 UNIT = "TFLOP/s"
 STEP_WORKLOAD = ("FLUX.1-dev 1024x1024 joint attention B1 H24 S4608 D128: Ulysses-8 exchange of Q/K/V, "
-                 "ring-8 blockwise attention (8 x 576 keys) + LSE merge, inverse exchange of O")
+                 "ring-8 blockwise attention (8 x 576 keys) merged by LSE, inverse exchange of O")
 
 
 def step_config(world: int, B: int, S: int, H: int, D: int, P: int, n_blocks: int, l2: str) -> dict:
@@ -213,9 +217,14 @@ def run_ours(args):
         torch.sum(flush_buf, dim=0, out=flush_sink)
     scale = w.scale
     flop = w.flop
-    launches_per_step = 1 + 1 + 1  # exchange of Q, K, V; attention; merge fused with the inverse exchange
+    launches_per_step = 1 + 1  # exchange of Q, K, V; ring attention with the merge and the inverse exchange
+    view = lambda t: t.view(Bp, S, Hp, D)  # noqa: E731  (head shards as one BSHD tensor)
 
     def step(evs=None, x=None, out=None):
+        """The hot path in two launches: the Ulysses exchange of Q, K and V, then ring
+        attention over the 8 K/V blocks on every head shard with the LSE merge carried in
+        TMEM from block to block and each finished row stored to its token-sharded place
+        (the inverse exchange), cp_ring_sim_fused_ulysses."""
         x = x or (xq, xk, xv)
         out = o_seq if out is None else out
         if evs:
@@ -223,16 +232,28 @@ def run_ours(args):
         binding.ulysses_permute_n(x, P, 0, dsts=(yq, yk, yv))
         if evs:
             evs[1].record()
-        view = lambda t: t.view(Bp, S, Hp, D)
+        binding.ring_sim_fused_ulysses(yq, yk, yv, P, bounds, scale=scale, out=out, out_lse=lse_full)
+        if evs:
+            evs[2].record()
+
+    def step3(evs=None):
+        """The same hot path in three launches, each block's fp32 partial and LSE written to
+        HBM: the exchange, blockwise attention over the 8 blocks, then the LSE merge writing
+        each merged row to its token-sharded place (cp_attn_merge_ulysses)."""
+        if evs:
+            evs[0].record()
+        binding.ulysses_permute_n((xq, xk, xv), P, 0, dsts=(yq, yk, yv))
+        if evs:
+            evs[1].record()
         binding.attn_fwd_blocks(view(yq), view(yk), view(yv), bounds, scale=scale, partials=parts, lses=lses)
         if evs:
             evs[2].record()
-        # The LSE merge writes each merged row straight to its sequence-sharded position: the
-        # merge and the second all-to-all in one pass (cp_attn_merge_ulysses).
-        binding.attn_merge_ulysses(parts, lses, P, out=out, out_lse=lse_full)
+        binding.attn_merge_ulysses(parts, lses, P, out=o_seq3, out_lse=lse3)
         if evs:
             evs[3].record()
 
+    o_seq3 = torch.empty_like(o_seq)
+    lse3 = torch.empty_like(lse_full)
     for _ in range(args.warmup):
         flush_l2()
         step()
@@ -241,7 +262,7 @@ def run_ours(args):
 
     clocks = ClockSampler(local)
     clocks.start()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -256,11 +277,26 @@ def run_ours(args):
     clocks.stop()
     assert binding.last_device_status() == 0, "device status not OK after timed region"
 
-    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    step_ms = [e[0].elapsed_time(e[2]) for e in evs]
     perm_ms = [e[0].elapsed_time(e[1]) for e in evs]
     attn_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    merge_ms = [e[2].elapsed_time(e[3]) for e in evs]
     total_ms = reduce_max(sum(step_ms), dev)
+
+    # The three-launch form, timed the same way (its merge is the merge kernel's number).
+    n3 = min(args.steps, 200)
+    for _ in range(max(args.warmup, 3)):
+        flush_l2()
+        step3()
+    evs3 = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n3)]
+    for i in range(n3):
+        flush_l2()
+        step3(evs3[i])
+    torch.cuda.synchronize()
+    assert binding.last_device_status() == 0
+    step3_ms = statistics.mean(e[0].elapsed_time(e[3]) for e in evs3)
+    perm3_ms = [e[0].elapsed_time(e[1]) for e in evs3]
+    attn3_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs3)
+    merge_ms = [e[2].elapsed_time(e[3]) for e in evs3]
 
     # Single-block attention (the FLUX ring-1 case) timed on its own.
     qd, kd, vd = (t.to(dev) for t in (q_h, k_h, v_h))
@@ -278,10 +314,9 @@ def run_ours(args):
     ring1_ms = statistics.mean(a.elapsed_time(b) for a, b in r1[max(args.warmup, 3):])
 
     # The ring with the LSE merge fused into the attention kernel (no partials, no merge
-    # pass), on the same head-sharded tensors as the step.
+    # pass), on the same head-sharded tensors as the step, head-sharded output.
     fo = torch.empty_like(o_h)
     fl = torch.empty_like(lse_h)
-    view = lambda t: t.view(Bp, S, Hp, D)
     rf = []
     for i in range(max(args.warmup, 3) + 50):
         flush_l2()
@@ -304,18 +339,6 @@ def run_ours(args):
             evs.append((a, b))
         torch.cuda.synchronize()
         return statistics.mean(a.elapsed_time(b) for a, b in evs[max(args.warmup, 3):])
-
-    # The step in two launches: the exchange of Q/K/V, then the ring with the LSE merge
-    # carried in TMEM across the blocks and the inverse exchange in the kernel's epilogue
-    # (cp_ring_sim_fused_ulysses): no fp32 partials and no merge pass.
-    o_seq2 = torch.empty_like(o_seq)
-    lse2 = torch.empty_like(lse_full)
-
-    def step2():
-        binding.ulysses_permute_n((xq, xk, xv), P, 0, dsts=(yq, yk, yv))
-        binding.ring_sim_fused_ulysses(yq, yk, yv, P, bounds, scale=scale, out=o_seq2, out_lse=lse2)
-
-    step2_ms = timed_ms(step2, reps=50)
 
     # Unified SP: Ulysses 2 x ring 4 and Ulysses 4 x ring 2 on the same tensors, through
     # cp_usp_sim (exchange, ring attention + merge, inverse exchange, LSE regroup).
@@ -445,7 +468,7 @@ def run_ours(args):
         perm_bytes = 3 * 2 * B * S * H * D * 2
         part_bytes = n_blocks * rows * (4 * D + 4)
         merge_gbs = merge_bytes / (statistics.mean(merge_ms) * 1e-3) / 1e9
-        perm_gbs = perm_bytes / (statistics.mean(perm_ms) * 1e-3) / 1e9
+        perm_gbs = perm_bytes / (statistics.mean(perm_ms + perm3_ms) * 1e-3) / 1e9
         line = {
             "metric": METRIC,
             "value": round(value, 2),
@@ -463,7 +486,7 @@ def run_ours(args):
             "config": step_config(world, B, S, H, D, P, n_blocks,
                                   "flushed between timed steps (read of %d MiB > L2)" % flush_mib),
             "roofline": {
-                "kernel": "attn_fwd_sm100 (8 ring blocks in one launch)",
+                "kernel": "attention, 8 ring blocks in one launch, merge in TMEM, inverse exchange in the epilogue",
                 "bound": "tensor",
                 "achieved": round(attn_tflops, 2),
                 "peak": peaks["bf16_tflops"],
@@ -480,12 +503,14 @@ def run_ours(args):
             "kernels": {
                 "attn_ring1_tflops": round(ring1_tflops, 2),
                 "attn_ring1_ms": round(ring1_ms, 4),
-                "attn_ring8_ms": round(attn_mean, 4),
+                "attn_ring8_fused_ulysses_ms": round(attn_mean, 4),
                 "ring8_fused_ms": round(fused_ms, 4),
                 "ring8_fused_tflops": round(flop / (fused_ms * 1e-3) / 1e12, 2),
+                "step_3launch_ms": round(step3_ms, 4),
+                "step_3launch_tflops": round(flop / (step3_ms * 1e-3) / 1e12, 2),
+                "attn_ring8_blocks_ms": round(attn3_ms, 4),
+                "attn_ring8_blocks_tflops": round(flop / (attn3_ms * 1e-3) / 1e12, 2),
                 "attn_ring8_partial_bytes": part_bytes,
-                "step_2launch_fused_ulysses_ms": round(step2_ms, 4),
-                "step_2launch_fused_ulysses_tflops": round(flop / (step2_ms * 1e-3) / 1e12, 2),
                 "merge_inverse_exchange_ms": round(statistics.mean(merge_ms), 4),
                 "merge_inverse_exchange_gbs": round(merge_gbs, 1),
                 "merge_inverse_exchange_frac_of_measured_hbm": round(merge_gbs / peaks["hbm_gbs"], 4),
@@ -623,6 +648,10 @@ def run_profile_case(args):
             binding.attn_fwd(q, k, v)
         elif case == "attn_ring8":
             binding.attn_fwd_blocks(q, k, v, bounds)
+        elif case == "attn_fused_ulysses":  # the step's attention: head shards in, token shards out
+            heads = [t.view(B, P, S // P, H, D).permute(1, 0, 2, 3, 4).contiguous() for t in (q, k, v)]
+            heads = binding.ulysses_permute_n(heads, P, 0)
+            binding.ring_sim_fused_ulysses(*heads, P, bounds)
         elif case == "merge":  # the step's merge: head-shard partials, fused with the inverse exchange
             parts = torch.randn(8, P * B, S, H // P, D, device="cuda")
             lses = torch.randn(8, P * B, H // P, S, device="cuda")
@@ -661,7 +690,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-budget", type=float, default=90.0)
-    ap.add_argument("--profile-case", choices=["attn_ring1", "attn_ring8", "merge", "permute", "push", "anything", "gather"], default=None)
+    ap.add_argument("--profile-case", choices=["attn_ring1", "attn_ring8", "attn_fused_ulysses", "merge", "permute", "push", "anything",
+                                                      "gather"], default=None)
     ap.add_argument("--profile-batch", type=int, default=2)
     ap.add_argument("--profile-reps", type=int, default=3)
     args = ap.parse_args()

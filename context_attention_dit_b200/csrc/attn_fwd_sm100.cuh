@@ -65,7 +65,9 @@ constexpr int kEpilogueWarp0 = 12;
 constexpr int kSoftmaxRegs = 136;
 constexpr int kControlRegs = 48;
 constexpr int kEpilogueRegs = 192;
-static_assert(2 * kSoftmaxRegs + kControlRegs + kEpilogueRegs == 4 * 128, "register split must use the launch budget");
+constexpr int kLaunchRegs = 65536 / kAttnThreads;  // registers per thread at launch (128)
+static_assert(2 * kSoftmaxRegs + kControlRegs + kEpilogueRegs == 4 * kLaunchRegs,
+              "register split must use the launch budget");
 static_assert(kSoftmaxRegs >= 128 && kEpilogueRegs >= 128 && kControlRegs <= 128,
               "softmax and epilogue warpgroups grow (setmaxnreg.inc), the control warps shrink");
 constexpr int kTmemCols = 512;
@@ -825,10 +827,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   // Producer and MMA roles run on lane 0 of their warp; the other lanes wait at the
   // __syncwarp so that each warp is converged again for the teardown below.
   if (warp >= kEpilogueWarp0) {
-    regs_increase<kEpilogueRegs>();
+    regs_set<kEpilogueRegs, kLaunchRegs>();
     attn_epilogue<D>(p, smem, bars, tmem, abort_flag);
   } else if (warp >= 8) {
-    regs_decrease<kControlRegs>();
+    regs_set<kControlRegs, kLaunchRegs>();
     if (warp == kProducerWarp) {
       if ((threadIdx.x & 31) == 0) attn_producer_qk<D>(&tm_q, &tm_k, p, smem, bars, abort_flag);
     } else if (warp == kVProducerWarp) {
@@ -840,7 +842,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     __syncwarp();
   } else {
-    regs_increase<kSoftmaxRegs>();
+    regs_set<kSoftmaxRegs, kLaunchRegs>();
     attn_softmax<D>(p, smem, bars, tmem, abort_flag);
   }
 

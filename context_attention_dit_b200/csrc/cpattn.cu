@@ -10,7 +10,6 @@
 #include <cmath>
 #include <cstdint>
 #include <algorithm>
-#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -18,7 +17,6 @@
 #include <nvtx3/nvToolsExt.h>
 
 #include "attn_fwd_sm100.cuh"
-#include "attn_pair_sm100.cuh"
 #include "lse_merge.cuh"
 #include "peer.cuh"
 #include "ring_gather.cuh"
@@ -40,18 +38,7 @@ struct DeviceInfo {
   int num_sms = 0;
   int* status = nullptr;  // device address of g_cp_status
   bool attn_attr_set[2] = {false, false};
-  bool pair_attr_set[2] = {false, false};
 };
-
-// Which attention kernel runs: the one-Q-tile kernel (attn_fwd_sm100) unless
-// CPATTN_ATTN_KERNEL=pair selects the two-Q-tile kernel (attn_pair_sm100).
-bool use_pair_kernel() {
-  static const bool pair = [] {
-    const char* e = std::getenv("CPATTN_ATTN_KERNEL");
-    return e && std::strcmp(e, "pair") == 0;
-  }();
-  return pair;
-}
 
 std::mutex g_mutex;
 DeviceInfo g_dev[kMaxDevices];
@@ -267,30 +254,6 @@ cp_status launch_attn(const void* q, const void* k, const void* v, const int* bo
       make_bshd_map(&tv, vp, B, Skv > 0 ? kv_rows : Sq, H, D, kvs) != CP_OK)
     return CP_ERR_CUDA;
 
-  if (use_pair_kernel()) {
-    const int units = B * H * ((p.n_qt + 1) / 2);
-    const int grid = units < dev->num_sms ? units : dev->num_sms;
-    if (D == 128) {
-      using L = pair::Smem<128>;
-      if (!dev->pair_attr_set[1]) {
-        if (cudaFuncSetAttribute(pair::attn_pair_sm100_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 L::kRequest) != cudaSuccess)
-          return CP_ERR_CUDA;
-        dev->pair_attr_set[1] = true;
-      }
-      pair::attn_pair_sm100_kernel<128><<<grid, pair::kThreads, L::kRequest, stream>>>(tq, tk, tv, p);
-    } else {
-      using L = pair::Smem<64>;
-      if (!dev->pair_attr_set[0]) {
-        if (cudaFuncSetAttribute(pair::attn_pair_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 L::kRequest) != cudaSuccess)
-          return CP_ERR_CUDA;
-        dev->pair_attr_set[0] = true;
-      }
-      pair::attn_pair_sm100_kernel<64><<<grid, pair::kThreads, L::kRequest, stream>>>(tq, tk, tv, p);
-    }
-    return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
-  }
   const int grid = p.n_units < dev->num_sms ? p.n_units : dev->num_sms;
   if (D == 128) {
     using L = AttnSmem<128>;
@@ -681,11 +644,9 @@ cp_status cp_ring_anything_gather(const void* const* srcs, void* const* dsts, in
     using V = decltype(tag);
     const int row_vecs = static_cast<int>(row_bytes / sizeof(V));
     const long long groups = (rows + kGatherRows - 1) / kGatherRows;
-    // About 8 resident blocks of rows per SM, each looping over its share of row groups.
-    const long long cap = static_cast<long long>(dev->num_sms) * 8;
     const dim3 grid((row_vecs + kGatherThreads - 1) / kGatherThreads,
-                    static_cast<unsigned>(std::min<long long>(groups, std::max<long long>(1, cap))), n_tensors);
-    ring_anything_gather_kernel<V><<<grid, kGatherThreads, 0, cs>>>(a, row_vecs, rows);
+                    static_cast<unsigned>(std::min<long long>(groups, 65535)), n_tensors);
+    ring_anything_gather_kernel<V><<<grid, kGatherThreads, 0, cs>>>(a, row_vecs, static_cast<int>(rows));
   };
   if (row_bytes % 16 == 0)
     launch(uint4{});

@@ -33,44 +33,43 @@ struct GatherArgs {
   int n_chunks, B, S, max_len;
 };
 
-// Source row of destination row R = (c * B + b) * max_len + r, or -1 for a padding row.
-__device__ __forceinline__ long long gather_src_row(const GatherArgs& a, long long R) {
-  const long long per_c = static_cast<long long>(a.B) * a.max_len;
-  const int c = static_cast<int>(R / per_c);
-  const long long rem = R - c * per_c;
-  const int b = static_cast<int>(rem / a.max_len);
-  const int r = static_cast<int>(rem - static_cast<long long>(b) * a.max_len);
-  if (r >= a.bounds[c + 1] - a.bounds[c]) return -1;
-  return static_cast<long long>(b) * a.S + a.bounds[c] + r;
-}
-
 template <typename V>
 __global__ void __launch_bounds__(kGatherThreads)
-    ring_anything_gather_kernel(const __grid_constant__ GatherArgs a, int row_vecs, long long rows) {
+    ring_anything_gather_kernel(const __grid_constant__ GatherArgs a, int row_vecs, int rows) {
   const int i = blockIdx.x * kGatherThreads + threadIdx.x;  // vector within the row
   if (i >= row_vecs) return;
   const V* __restrict__ src = static_cast<const V*>(a.src[blockIdx.z]);
   V* __restrict__ dst = static_cast<V*>(a.dst[blockIdx.z]);
   const long long src_total = static_cast<long long>(a.B) * a.S * row_vecs;
-  const long long dst_total = rows * row_vecs;
-  for (long long R0 = static_cast<long long>(blockIdx.y) * kGatherRows; R0 < rows;
-       R0 += static_cast<long long>(gridDim.y) * kGatherRows) {
+  const long long dst_total = static_cast<long long>(rows) * row_vecs;
+  const int per_c = a.B * a.max_len;  // destination rows per block
+  for (int R0 = blockIdx.y * kGatherRows; R0 < rows; R0 += gridDim.y * kGatherRows) {
+    // Destination row R = (c * B + b) * max_len + r; the rows of a group are consecutive,
+    // so (c, b, r) is found once and stepped.
+    int c = R0 / per_c;
+    const int rem = R0 - c * per_c;
+    int b = rem / a.max_len;
+    int r = rem - b * a.max_len;
     V v[kGatherRows];
 #pragma unroll
     for (int k = 0; k < kGatherRows; ++k) {
       v[k] = V{};
-      const long long R = R0 + k;
-      if (R < rows) {
-        const long long sr = gather_src_row(a, R);
-        const long long si = sr * row_vecs + i;
-        if (sr >= 0 && in_bounds(si, 1, src_total)) v[k] = src[si];
+      if (R0 + k < rows && r < a.bounds[c + 1] - a.bounds[c]) {  // a true row of block c, else padding
+        const long long si = (static_cast<long long>(b) * a.S + a.bounds[c] + r) * row_vecs + i;
+        if (in_bounds(si, 1, src_total)) v[k] = src[si];
+      }
+      if (++r == a.max_len) {
+        r = 0;
+        if (++b == a.B) {
+          b = 0;
+          ++c;
+        }
       }
     }
 #pragma unroll
     for (int k = 0; k < kGatherRows; ++k) {
-      const long long R = R0 + k;
-      const long long di = R * row_vecs + i;
-      if (R < rows && in_bounds(di, 1, dst_total)) dst[di] = v[k];
+      const long long di = static_cast<long long>(R0 + k) * row_vecs + i;
+      if (R0 + k < rows && in_bounds(di, 1, dst_total)) dst[di] = v[k];
     }
   }
 }
