@@ -47,14 +47,15 @@ def step_config(world: int, B: int, S: int, H: int, D: int, P: int, n_blocks: in
             "ulysses_degree": P, "ring_degree": n_blocks,
             "parallelism": f"replicas x{world} (single-GPU simulated degrees)", "l2": l2}
 
-# DRAM traffic of the timed attention launch (8 ring blocks, FLUX B1), from one ncu capture
-# of the same kernel on the B2 shape (profiles/attn_fwd_sm100__flux_b2_ring8.md):
-# dram__bytes_read.sum + dram__bytes_write.sum = 186.38 + 860.91 MB, halved to one B1 launch
-# (the B1 launch processes half the units; Q/K/V reads and partial writes scale with them).
+# DRAM traffic of the timed attention launch (the fused ring over 8 blocks with the Ulysses
+# output map, FLUX B1), from one ncu capture of the same kernel on the B2 shape
+# (profiles/attn_fwd_sm100__flux_b2_ring8_fused_ulysses.md):
+# dram__bytes_read.sum + dram__bytes_write.sum = 169.97 + 40.27 MB, halved to one B1 launch
+# (the B1 launch processes half the units; Q/K/V reads and output writes scale with them).
 # It describes only the kernel source it was captured on, identified by its SHA-256.
 ATTN_TRAFFIC = {
-    "kernel_sha256": "7f9867163754f9086e8eed92df542cb8c6d4fe4094ee51cb2303033950e6006a",
-    "bytes_per_launch": (186_379_776 + 860_907_008) // 2,
+    "kernel_sha256": "998b54a6dfcb46a411c7ec945cd6171945e28a135347b12e9e57b41e6455baf3",
+    "bytes_per_launch": (169_971_712 + 40_270_080) // 2,
 }
 
 
@@ -297,6 +298,19 @@ def run_ours(args):
     perm3_ms = [e[0].elapsed_time(e[1]) for e in evs3]
     attn3_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs3)
     merge_ms = [e[2].elapsed_time(e[3]) for e in evs3]
+    # The merge on its own: inside the step it follows the attention launch, whose last
+    # ~100 MB of partials are still dirty in L2 and are written back while the merge runs.
+    # Here the partials of the last step are in HBM and L2 is flushed before each merge.
+    iso = []
+    for i in range(max(args.warmup, 3) + 50):
+        flush_l2()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        binding.attn_merge_ulysses(parts, lses, P, out=o_seq3, out_lse=lse3)
+        b.record()
+        iso.append((a, b))
+    torch.cuda.synchronize()
+    merge_iso_ms = statistics.mean(a.elapsed_time(b) for a, b in iso[max(args.warmup, 3):])
 
     # Single-block attention (the FLUX ring-1 case) timed on its own.
     qd, kd, vd = (t.to(dev) for t in (q_h, k_h, v_h))
@@ -468,6 +482,7 @@ def run_ours(args):
         perm_bytes = 3 * 2 * B * S * H * D * 2
         part_bytes = n_blocks * rows * (4 * D + 4)
         merge_gbs = merge_bytes / (statistics.mean(merge_ms) * 1e-3) / 1e9
+        merge_iso_gbs = merge_bytes / (merge_iso_ms * 1e-3) / 1e9
         perm_gbs = perm_bytes / (statistics.mean(perm_ms + perm3_ms) * 1e-3) / 1e9
         line = {
             "metric": METRIC,
@@ -511,10 +526,12 @@ def run_ours(args):
                 "attn_ring8_blocks_ms": round(attn3_ms, 4),
                 "attn_ring8_blocks_tflops": round(flop / (attn3_ms * 1e-3) / 1e12, 2),
                 "attn_ring8_partial_bytes": part_bytes,
-                "merge_inverse_exchange_ms": round(statistics.mean(merge_ms), 4),
-                "merge_inverse_exchange_gbs": round(merge_gbs, 1),
-                "merge_inverse_exchange_frac_of_measured_hbm": round(merge_gbs / peaks["hbm_gbs"], 4),
-                "merge_inverse_exchange_frac_of_spec_8000": round(merge_gbs / 8000.0, 4),
+                "merge_inverse_exchange_ms": round(merge_iso_ms, 4),
+                "merge_inverse_exchange_gbs": round(merge_iso_gbs, 1),
+                "merge_inverse_exchange_frac_of_measured_hbm": round(merge_iso_gbs / peaks["hbm_gbs"], 4),
+                "merge_inverse_exchange_frac_of_spec_8000": round(merge_iso_gbs / 8000.0, 4),
+                "merge_inverse_exchange_in_3launch_step_ms": round(statistics.mean(merge_ms), 4),
+                "merge_inverse_exchange_in_3launch_step_gbs": round(merge_gbs, 1),
                 "permute_qkv_ms": round(statistics.mean(perm_ms), 4),
                 "permute_qkv_gbs": round(perm_gbs, 1),
                 "permute_qkv_frac_of_measured_hbm": round(perm_gbs / peaks["hbm_gbs"], 4),
