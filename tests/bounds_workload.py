@@ -42,6 +42,20 @@ def run():
     qs, ks, vs = (t.cuda() for t in make_qkv(1, 4, 8128, 300, 128, seed=10))
     assert binding.ring_workspace_size(2, 1, 4, 8128, 128) > binding.STATIC_SCRATCH_BYTES - 4096
     record("ring_static_near_limit", *binding.ring_sim_static(qs, ks, vs, [0, 150, 300]))
+    # Views: a K/V block inside a longer sequence, an output written into a larger tensor,
+    # and the fused ring writing the Ulysses token-sharded layout.
+    qv, kv_full, vv_full = (t.cuda() for t in make_qkv(2, 3, 200, 700, 128, seed=11))
+    big = torch.zeros(2, 210, 3, 128, dtype=torch.bfloat16, device="cuda")
+    binding.attn_fwd_strided(qv, kv_full[:, 123:600], vv_full[:, 123:600], out=big[:, 5:205])
+    record("attn_strided", big)
+    Pu, Bu, Su, Hu = 2, 2, 256, 4
+    xs = [t.reshape(Bu, Pu, Su // Pu, Hu, 64).permute(1, 0, 2, 3, 4).contiguous().cuda()
+          for t in make_qkv(Bu, Hu, Su, Su, 64, seed=12)]
+    heads = binding.ulysses_permute_n(xs, Pu, 0)
+    record("fused_ulysses", *binding.ring_sim_fused_ulysses(*heads, Pu, [0, 100, 101, 256]))
+    # The Ring Anything gather with an empty block and padding.
+    gk = binding.ring_anything_gather([kv_full.contiguous()], [0, 0, 301, 700], 410)
+    record("gather", *gk)
     P, B, S, H, D = 4, 2, 384, 8, 128
     x = [t.cuda() for t in make_qkv(P * B, H // P, S, S, D, seed=5)]
     parts, lses = binding.attn_fwd_blocks(*x, [0, 100, 101, 384])

@@ -59,6 +59,15 @@ def test_packed_qkv_and_strided_output():
     assert torch.equal(big[:, 5:5 + S], o_d) and torch.equal(lse, lse_d)
 
 
+def test_empty_kv_view():
+    """A K/V block of no rows (an empty slice): O = 0 and lse = -inf, as with cp_attn_fwd."""
+    q, k_full, v_full = cuda(*qkv(2, 3, 77, 100, 64, seed=75))
+    o, lse = binding.attn_fwd_strided(q, k_full[:, 40:40], v_full[:, 40:40], out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert binding.last_device_status() == 0
+    assert torch.equal(o, torch.zeros_like(o)) and bool(torch.isneginf(lse).all())
+
+
 def test_interleaved_output_layout():
     """An output whose batches sit side by side within each sequence row ([S][B][H][D])."""
     B, S, H, D = 3, 200, 2, 64
@@ -87,12 +96,13 @@ def unshard(x):
     (2, 8, 384, 128, 4, [0, 128, 129, 384]),
     (1, 4, 200, 128, 2, [0, 0, 77, 200]),
 ])
-def test_fused_ulysses_small_matches_oracle(B, H, S, D, P, bounds):
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32], ids=["bf16", "fp32"])
+def test_fused_ulysses_small_matches_oracle(B, H, S, D, P, bounds, out_dtype):
     q, k, v = qkv(B, H, S, S, D, seed=74)
     scale = 1 / math.sqrt(D)
     o_ref, lse_ref = oracle.attention(q, k, v, scale)
     heads = binding.ulysses_permute_n([shard(t, P).cuda() for t in (q, k, v)], P, 0)
-    o, lse = binding.ring_sim_fused_ulysses(*heads, P, bounds, scale=scale)
+    o, lse = binding.ring_sim_fused_ulysses(*heads, P, bounds, scale=scale, out_dtype=out_dtype)
     torch.cuda.synchronize()
     assert binding.last_device_status() == 0
     assert o.shape == (P, B, S // P, H, D) and lse.shape == (B, H, S)
@@ -100,7 +110,7 @@ def test_fused_ulysses_small_matches_oracle(B, H, S, D, P, bounds):
     # The fused kernel with a plain output, followed by the inverse exchange, gives the same
     # bits: only the output address differs.
     view = lambda t: t.view(P * B, S, H // P, D)  # noqa: E731
-    of, lf = binding.ring_sim_fused(*(view(t) for t in heads), bounds, scale=scale)
+    of, lf = binding.ring_sim_fused(*(view(t) for t in heads), bounds, scale=scale, out_dtype=out_dtype)
     assert torch.equal(o, binding.ulysses_permute(of.view(P, B, S, H // P, D), P, 1))
     assert torch.equal(lse, lf.view(P, B, H // P, S).permute(1, 0, 2, 3).reshape(B, H, S))
 
