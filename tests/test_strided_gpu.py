@@ -134,3 +134,22 @@ def test_fused_ulysses_rejects_indivisible():
     x = torch.zeros(3, 1, 16, 2, 64, dtype=torch.bfloat16, device="cuda")  # S = 16 not divisible by 3
     with pytest.raises(ValueError):
         binding.ring_sim_fused_ulysses(x, x, x, 3, [0, 16])
+
+
+def test_fused_ulysses_video_sampled_rows():
+    """Video DiT (B1 H40 S32760 D128) over Ulysses-8 (5 heads per shard) x ring-4: sampled
+    rows against the fp64 oracle, every element against unsplit GPU attention."""
+    from tests.gpu_util import sample_rows
+
+    w, (q, k, v) = workload_inputs("video_s32760_ring4")
+    P, bounds = 8, even_bounds(w.S, 4)
+    rows = sample_rows(w.S, bounds + [i * w.S // P for i in range(P + 1)], n_random=200)
+    o_ref, lse_ref = oracle.attention_rows(q, k, v, w.scale, rows)
+    heads = binding.ulysses_permute_n([shard(t, P).cuda() for t in (q, k, v)], P, 0)
+    o, lse = binding.ring_sim_fused_ulysses(*heads, P, bounds, scale=w.scale)
+    torch.cuda.synchronize()
+    assert binding.last_device_status() == 0
+    o = unshard(o)
+    assert_attn_close(o[:, rows], lse[:, :, rows], o_ref, lse_ref, "video fused ulysses-8 x ring-4 (sampled rows)")
+    o1, _ = binding.attn_fwd(*cuda(q, k, v), scale=w.scale)
+    assert_split_close(o, o1, "video fused ulysses-8 x ring-4 vs unsplit")
