@@ -219,6 +219,9 @@ def attn_fwd_strided(q, k, v, scale: Optional[float] = None, out_dtype=torch.bfl
     o_sb, o_ss = _check_view("out", out)
     if lse is None and want_lse:
         lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
+    if lse is not None and (lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, Sq) or not lse.is_contiguous()
+                            or lse.device != q.device):
+        raise ValueError(f"lse must be a contiguous float32 tensor of shape {(B, H, Sq)}")
     st = load().cp_attn_fwd_strided(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Sq, Skv, D, q_sb, q_ss,
                                     kv_sb, kv_ss, o_sb, o_ss, scale, code, ctypes.c_void_p(_stream(q)))
     _check(st, "cp_attn_fwd_strided")
@@ -411,6 +414,12 @@ def ring_sim_fused_ulysses(q, k, v, degree: int, chunk_bounds: Sequence[int], sc
         out = torch.empty((P, B, S // P, H, D), dtype=out_dtype, device=q.device)
     if out_lse is None:
         out_lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    if out.dtype != out_dtype or tuple(out.shape) != (P, B, S // P, H, D) or not out.is_contiguous() \
+            or out.device != q.device:
+        raise ValueError(f"out must be a contiguous {out_dtype} tensor of shape {(P, B, S // P, H, D)}")
+    if out_lse.dtype != torch.float32 or tuple(out_lse.shape) != (B, H, S) or not out_lse.is_contiguous() \
+            or out_lse.device != q.device:
+        raise ValueError(f"out_lse must be a contiguous float32 tensor of shape {(B, H, S)}")
     st = load().cp_ring_sim_fused_ulysses(_ptr(q), _ptr(k), _ptr(v), P, bounds, n, _ptr(out), _ptr(out_lse), B, S, H,
                                           D, scale, code, ctypes.c_void_p(_stream(q)))
     _check(st, "cp_ring_sim_fused_ulysses")
@@ -441,6 +450,13 @@ def ring_anything_gather(srcs, chunk_bounds: Sequence[int], max_len: Optional[in
     if dsts is None:
         dsts = [torch.empty((n, B, max_len, H, D), dtype=ref.dtype, device=ref.device) for _ in srcs]
     dsts = list(dsts)
+    if len(dsts) != len(srcs):
+        raise ValueError(f"{len(srcs)} sources but {len(dsts)} destinations")
+    for d in dsts:
+        if not isinstance(d, torch.Tensor) or not d.is_cuda or not d.is_contiguous() or d.dtype != ref.dtype \
+                or d.device != ref.device or d.numel() != n * B * max_len * H * D:
+            raise ValueError(f"destinations must be contiguous CUDA tensors of {ref.dtype} with "
+                             f"{n}*{B}*{max_len}*{H}*{D} elements on {ref.device}")
     cnt = len(srcs)
     sp = (ctypes.c_void_p * cnt)(*[t.data_ptr() for t in srcs])
     dp = (ctypes.c_void_p * cnt)(*[t.data_ptr() for t in dsts])

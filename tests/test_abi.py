@@ -397,3 +397,17 @@ def test_ring_anything_gather_checks_before_cuda(lib):
     assert call(srcs, (vp * 2)(3 << 20, 3 << 20), 2, (0, 3, 5), 3) == I.CP_ERR_INVALID_ARG  # dsts overlap
     assert call(srcs, (vp * 2)(3 << 20, (4 << 20) + 8), 2, (0, 3, 5), 3) == I.CP_ERR_MISALIGNED
     assert call(srcs, dsts, 2, (0, 0, 0), 0) == I.CP_OK                   # no rows: nothing to copy
+
+
+def test_new_bindings_reject_bad_outputs_before_the_library():
+    """The Python side of the strided, fused-Ulysses and gather calls checks the tensors it
+    is given (host tensors and wrong shapes never reach the library)."""
+    import torch
+
+    with pytest.raises(ValueError):
+        binding.attn_fwd_strided(torch.zeros(1, 4, 2, 64, dtype=torch.bfloat16), torch.zeros(1, 4, 2, 64, dtype=torch.bfloat16),
+                                 torch.zeros(1, 4, 2, 64, dtype=torch.bfloat16))  # host tensors
+    with pytest.raises(ValueError):
+        binding.ring_sim_fused_ulysses(*(torch.zeros(2, 1, 8, 2, 64, dtype=torch.bfloat16) for _ in range(3)), 2, [0, 8])
+    with pytest.raises(ValueError):
+        binding.ring_anything_gather([torch.zeros(1, 5, 1, 8, dtype=torch.bfloat16)], [0, 2, 5])  # host source
