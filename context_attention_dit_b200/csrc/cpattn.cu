@@ -194,6 +194,17 @@ cp_status launch_attn(const void* q, const void* k, const void* v, const int* bo
     dl.o = dense(Sq, H, D);
     lay = &dl;
   }
+  // Fused: every block feeds one running softmax, and the blocks are consecutive ranges of
+  // one K/V tensor, so their union is tiled as one range.  A 128-key tile may then hold the
+  // end of one block and the start of the next, and a block no longer ends in a short tile
+  // (576-key ring-8 blocks would otherwise cost 5 tiles each instead of 4.5).
+  int union_bounds[2];
+  if (fuse && n_chunks > 1) {
+    union_bounds[0] = bounds[0];
+    union_bounds[1] = bounds[n_chunks];
+    bounds = union_bounds;
+    n_chunks = 1;
+  }
   AttnParams p;
   std::memset(&p, 0, sizeof(p));
   p.B = B;

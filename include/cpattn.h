@@ -182,8 +182,9 @@ CP_API cp_status cp_ring_sim(const void* q, const void* k, const void* v, const 
  * queries meet the K/V blocks one after another and accumulate the result.  Here the
  * running (max, sum, output) of each query row is carried in TMEM from one block to the
  * next inside one launch, so no per-block partial is written and no merge pass runs; the
- * result equals merging the per-block partials (up to fp32 rounding order).  Key tiles
- * still end at block bounds, as in the unfused path.
+ * result equals merging the per-block partials (up to fp32 rounding order).  The blocks
+ * are consecutive ranges of one K/V tensor feeding one running softmax, so the kernel tiles
+ * their union: a 128-key tile may hold the end of one block and the start of the next.
  * Arguments as cp_ring_sim without the workspace; allocates nothing.  Output and LSE as
  * cp_attn_fwd; an all-empty split gives out = 0, lse = -inf.
  */
