@@ -6,8 +6,9 @@ the host orchestration run exactly as with one GPU per rank.  The barriers are t
 host's (stream synchronise + the gloo group's barrier): device-side barriers of ranks
 that share one GPU would be kernels waiting on one another, which these tests never
 launch.  Every rank's output is compared bit for bit with the single-process path on
-the unsplit tensors (``attn_fwd`` for Ulysses alone, ``ring_sim`` over the ring's
-blocks otherwise), and a small case also with the fp64 oracle.
+the unsplit tensors (``attn_fwd`` for Ulysses alone; otherwise, as each rank computes it,
+``attn_fwd`` of every ring block into an fp32 partial and ``attn_merge`` of the partials),
+and a small case also with the fp64 oracle.
 """
 
 import os
@@ -66,7 +67,13 @@ def _rank_main(rank, world, port, cfg, out_q):
                 bounds = [0]
                 for n in blk:
                     bounds.append(bounds[-1] + n)
-                ref, _, _ = binding.ring_sim(qc, kc, vc, bounds)
+                parts, lses = [], []
+                for c in range(R):
+                    kb, vb = (x[:, bounds[c]:bounds[c + 1]].contiguous() for x in (kc, vc))
+                    o_c, l_c = binding.attn_fwd(qc, kb, vb, out_dtype=torch.float32)
+                    parts.append(o_c)
+                    lses.append(l_c)
+                ref, _ = binding.attn_merge(torch.stack(parts), torch.stack(lses))
             ref = ref.cpu()
             result = {"status": status}
             for it in range(2):

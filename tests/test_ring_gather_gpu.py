@@ -10,7 +10,7 @@ import torch
 import oracle
 from context_attention_dit_b200 import binding
 from context_attention_dit_b200.inputs import make_qkv
-from tests.gpu_util import assert_attn_close, cuda, qkv
+from tests.gpu_util import LSE_ABS, assert_attn_close, assert_split_close, cuda, qkv
 
 pytestmark = pytest.mark.gpu
 
@@ -40,7 +40,9 @@ def test_gather_bit_exact(B, S, H, D, bounds, max_len, dtype):
 
 def test_ring_over_sliced_blocks_equals_ring_sim():
     """Attention of every true-length slice of the gathered K/V (strided views, no copy),
-    merged by LSE: the same tiles and arithmetic as cp_ring_sim, so the same bits."""
+    merged by LSE: the same launches and arithmetic as attention of each block cut from the
+    unpadded K/V, so the same bits; and the same result as cp_ring_sim (which runs every
+    block in one launch) up to fp32 rounding order."""
     B, H, S, D = 2, 4, 4481, 128
     bounds = binding.ring_bounds(S, 4, anything=True)      # 1121/1120/1120/1120
     q, k, v = cuda(*make_qkv(B, H, S, S, D, seed=82, rms_norm_qk=True))
@@ -53,10 +55,16 @@ def test_ring_over_sliced_blocks_equals_ring_sim():
         L = bounds[c + 1] - bounds[c]
         binding.attn_fwd_strided(q, gk[c, :, :L], gv[c, :, :L], out_dtype=torch.float32, out=parts[c], lse=lses[c])
     o, lse = binding.attn_merge(parts, lses)
-    ref, ref_lse, _ = binding.ring_sim(q, k, v, bounds)
+    for c in range(n):
+        kb, vb = (x[:, bounds[c]:bounds[c + 1]].contiguous() for x in (k, v))
+        binding.attn_fwd(q, kb, vb, out_dtype=torch.float32, out=parts[c], lse=lses[c])
+    ref, ref_lse = binding.attn_merge(parts, lses)
+    o_ring, lse_ring, _ = binding.ring_sim(q, k, v, bounds)
     torch.cuda.synchronize()
     assert binding.last_device_status() == 0
     assert torch.equal(o, ref) and torch.equal(lse, ref_lse)
+    assert_split_close(o, o_ring, "sliced gathered blocks vs cp_ring_sim")
+    assert float((lse - lse_ring).abs().max()) <= LSE_ABS
 
 
 def test_ring_over_sliced_blocks_matches_oracle():
