@@ -170,6 +170,29 @@ def test_fused_ring_matches_oracle_and_unfused(shape, bounds):
     assert_split_close(o, o2, f"fused vs unfused {bounds}")
 
 
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32], ids=["bf16", "fp32"])
+@pytest.mark.parametrize(
+    "shape,bounds",
+    [
+        ((1, 24, 4608, 4608, 128), [576 * i for i in range(9)]),  # FLUX ring-8
+        ((2, 3, 300, 300, 128), [0, 100, 200, 300]),
+        ((1, 2, 200, 450, 64), [0, 0, 130, 130, 450]),          # empty blocks
+        ((1, 2, 129, 17, 64), [0, 5, 6, 17]),
+    ],
+)
+def test_fused_ring_equals_unsplit_bit_for_bit(shape, bounds, out_dtype):
+    """The fused ring's blocks are consecutive ranges of one K/V tensor feeding one running
+    softmax, so the launch tiles their union exactly as unsplit attention tiles the keys:
+    the result does not depend on the split at all, bit for bit."""
+    B, H, Sq, Skv, D = shape
+    q, k, v = cuda(*qkv(B, H, Sq, Skv, D, seed=47, rms=True))
+    o, lse = binding.ring_sim_fused(q, k, v, bounds, out_dtype=out_dtype)
+    o1, l1 = binding.attn_fwd(q, k, v, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    assert binding.last_device_status() == 0
+    assert torch.equal(o, o1) and torch.equal(lse, l1)
+
+
 def test_fused_ring_all_blocks_empty():
     q, k, v = cuda(*qkv(1, 2, 130, 0, 128))
     o, lse = binding.ring_sim_fused(q, k, v, [0, 0, 0])
