@@ -294,8 +294,11 @@ cp_status launch_merge(const float* partials, const float* lses, int n, void* ou
   const long long rows = static_cast<long long>(B) * H * Sq;
   const long long part_stride = rows * D;
   const long long lse_stride = rows;
-  // ST query positions per block (all heads), about 128 rows per block.
-  const int ST = H >= 128 ? 1 : (128 / H > 64 ? 64 : 128 / H);
+  // ST query positions per block (all heads), about 64 rows per block.  Blocks of about 128
+  // rows fit the FLUX merges in one wave whose blocks all stall on their LSE staging at once
+  // (24 heads: 3.6 TB/s); with 64 the second wave's staging overlaps the first wave's
+  // streaming (5.1 TB/s; 5.9 for the 3-head Ulysses shards).
+  const int ST = H >= 64 ? 1 : 64 / H;
   const long long gx = (Sq + ST - 1) / ST;
   if (B > 65535 || gx >= (1LL << 31)) return CP_ERR_UNSUPPORTED;
   const size_t smem = static_cast<size_t>(n) * H * ST * sizeof(float);
