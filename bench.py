@@ -50,12 +50,12 @@ def step_config(world: int, B: int, S: int, H: int, D: int, P: int, n_blocks: in
 # DRAM traffic of the timed attention launch (the fused ring over 8 blocks with the Ulysses
 # output map, FLUX B1), from one ncu capture of the same kernel on the B2 shape
 # (profiles/attn_fwd_sm100__flux_b2_ring8_fused_ulysses.md):
-# dram__bytes_read.sum + dram__bytes_write.sum = 170.01 + 39.31 MB, halved to one B1 launch
+# dram__bytes_read.sum + dram__bytes_write.sum = 169.96 + 43.90 MB, halved to one B1 launch
 # (the B1 launch processes half the units; Q/K/V reads and output writes scale with them).
 # It describes only the kernel source it was captured on, identified by its SHA-256.
 ATTN_TRAFFIC = {
-    "kernel_sha256": "998b54a6dfcb46a411c7ec945cd6171945e28a135347b12e9e57b41e6455baf3",
-    "bytes_per_launch": (170_006_272 + 39_311_360) // 2,
+    "kernel_sha256": "96aa2b09ae7037d97cfbd2edf9061b75e74a772e14ff93a248fb5e517b36cdf5",
+    "bytes_per_launch": (169_955_072 + 43_901_952) // 2,
 }
 
 

@@ -823,6 +823,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Launched as a programmatic dependent of the previous kernel in the stream: the setup
+  // above overlaps that kernel's tail; no global memory is read or written before it has
+  // completed and its writes are visible.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // Producer and MMA roles run on lane 0 of their warp; the other lanes wait at the
   // __syncwarp so that each warp is converged again for the teardown below.

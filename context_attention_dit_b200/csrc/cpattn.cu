@@ -178,6 +178,24 @@ struct AttnLayout {
   int uly_b = 0;
 };
 
+// The attention kernel launched as a programmatic dependent of the stream's previous kernel
+// (its prologue overlaps that kernel's tail; it waits for it before touching memory).
+template <typename Kernel>
+void launch_pdl(Kernel kernel, int grid, int smem, cudaStream_t stream, const CUtensorMap& tq, const CUtensorMap& tk,
+                const CUtensorMap& tv, const AttnParams& p) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kAttnThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, kernel, tq, tk, tv, p);
+}
+
 // Launch the attention kernel over n_chunks K/V blocks given by `bounds` (host array).
 // `lay` == nullptr: Q, K, V and the output are dense BSHD tensors.
 cp_status launch_attn(const void* q, const void* k, const void* v, const int* bounds, int n_chunks, void* out,
@@ -274,7 +292,7 @@ cp_status launch_attn(const void* q, const void* k, const void* v, const int* bo
         return CP_ERR_CUDA;
       dev->attn_attr_set[1] = true;
     }
-    attn_fwd_sm100_kernel<128><<<grid, kAttnThreads, L::kRequest, stream>>>(tq, tk, tv, p);
+    launch_pdl(attn_fwd_sm100_kernel<128>, grid, L::kRequest, stream, tq, tk, tv, p);
   } else {
     using L = AttnSmem<64>;
     if (!dev->attn_attr_set[0]) {
@@ -283,7 +301,7 @@ cp_status launch_attn(const void* q, const void* k, const void* v, const int* bo
         return CP_ERR_CUDA;
       dev->attn_attr_set[0] = true;
     }
-    attn_fwd_sm100_kernel<64><<<grid, kAttnThreads, L::kRequest, stream>>>(tq, tk, tv, p);
+    launch_pdl(attn_fwd_sm100_kernel<64>, grid, L::kRequest, stream, tq, tk, tv, p);
   }
   return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
 }
