@@ -146,3 +146,33 @@ def test_output_only_16_byte_aligned(out_dtype):
     binding.attn_fwd(*cuda(q, k, v), out_dtype=out_dtype, out=out)
     torch.cuda.synchronize()
     assert_attn_close(out, None, o_ref, lse_ref, "16-byte aligned output")
+
+
+def test_launch_orders_after_the_previous_kernel():
+    """The attention kernel is a programmatic dependent launch: its setup may overlap the
+    stream's previous kernel, but it must read inputs that kernel has just written and must
+    not overwrite a buffer that kernel is still reading."""
+    B, H, S, D = 1, 24, 4608, 128
+    q0, k, v = cuda(*qkv(B, H, S, S, D, seed=91, rms=True))
+    q1 = cuda(*qkv(B, H, S, S, D, seed=92, rms=True))[0]
+    want1, lse1 = binding.attn_fwd(q1, k, v)
+    want0, _ = binding.attn_fwd(q0, k, v)
+    out = torch.empty_like(q0)
+    lse = torch.empty_like(lse1)
+    torch.cuda.synchronize()
+    for _ in range(3):
+        # read after write: a copy kernel overwrites Q right before the launch
+        q = q0.clone()
+        torch.cuda.synchronize()
+        q.copy_(q1)
+        binding.attn_fwd(q, k, v, out=out, lse=lse)
+        torch.cuda.synchronize()
+        assert torch.equal(out, want1) and torch.equal(lse, lse1)
+        # write after read: a reduction reads the previous output right before the launch
+        binding.attn_fwd(q0, k, v, out=out)
+        total = out.sum(dtype=torch.float32)  # one reduction kernel reading want0's values
+        binding.attn_fwd(q1, k, v, out=out, lse=lse)
+        torch.cuda.synchronize()
+        assert torch.equal(total, want0.sum(dtype=torch.float32))
+        assert torch.equal(out, want1)
+    assert binding.last_device_status() == 0
